@@ -1,0 +1,580 @@
+#!/usr/bin/env python
+"""Benchmark of the column-sparse cross-step delta hot path on B200.
+
+One step is one sparse-delta step of a FLUX.1-dev-shaped DiT layer (1280x768
+image = 3840 + 512 text tokens, d_model 3072, MLP hidden 12288, 24 heads x
+128): the MLP delta (gathered up-projection with GELU / delta / cache
+writeback, then the gathered sparse-K down-projection into the fp32 output
+cache; 70% column sparsity, k = 3686 per 128-token block) and the attention
+delta (top 16.5% keys per 128-query block, k = 718, merged with the cached
+complement partial). Selections and caches come from a dense refresh of the
+previous step run with the same library. Steps alternate between two drifted
+inputs so every step changes the caches.
+
+Printed: one JSON line (rank 0). ``value`` is microseconds per layer-step for
+the whole job (max over ranks / number of GPUs); the other hot-path rows (top-k,
+dense refresh, cache gather / scatter, dense layer at k = all) are timed in
+the same run and reported under ``rows``.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample of
+the same workload, extrapolated to one layer-step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs/layer & useful TFLOP/s (% B200 bf16 peak) for sparse-delta MLP/attn"
+UNIT = "us/layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# FLUX.1-dev at 1280x768: 80x48 latent patches (2x2) = 3840 image tokens + 512 text tokens
+W = dict(T=4352, D=3072, H=12288, heads=24, d=128, Bt=128, mlp_permille=300, attn_permille=165, sigma=0.03)
+
+
+def k_of(n, permille):
+    return n * permille // 1000
+
+
+def flops_step(w):
+    """Useful FLOPs of one sparse step: selected columns / keys only."""
+    T, D, kc = w["T"], w["D"], k_of(w["H"], w["mlp_permille"])
+    kk = k_of(w["T"], w["attn_permille"])
+    up = 2 * T * D * kc
+    down = 2 * T * kc * D
+    attn = 4 * T * kk * w["d"] * w["heads"]
+    return up, down, attn
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS if k in p}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[1]) for r in rows]
+        mx = [num(r[2]) for r in rows]
+        pw = [num(r[3]) for r in rows]
+        loaded = [s for s, p in zip(sm, pw) if p > 250.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded), "power_w_max": max(pw)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+class OracleSample:
+    """A bounded sample of one layer-step for the fp64 CPU oracle: the MLP delta
+    on ``mlp_blocks`` token blocks and the attention delta on ``attn_tiles``
+    (head, query-block) tiles, with seeded synthetic inputs of the layer's
+    shapes. ``time_step`` runs it once and extrapolates linearly to the layer."""
+
+    def __init__(self, w, seed=0, mlp_blocks=8, attn_tiles=96):
+        import numpy as np
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+        except Exception:  # noqa: BLE001
+            self.cores = os.cpu_count() or 1
+        g = np.random.default_rng(seed)
+        T, D, H, h, d, Bt = w["T"], w["D"], w["H"], w["heads"], w["d"], w["Bt"]
+        self.w, self.nb = w, (T + Bt - 1) // Bt
+        kc, kk = k_of(H, w["mlp_permille"]), k_of(T, w["attn_permille"])
+        self.mlp_blocks = mlp_blocks
+        rows = mlp_blocks * Bt
+        self.x = g.standard_normal((rows, D))
+        self.W1 = g.standard_normal((D, H)) / math.sqrt(D)
+        self.b1 = 0.02 * g.standard_normal(H)
+        self.W2 = g.standard_normal((H, D)) / math.sqrt(H)
+        self.A = np.abs(g.standard_normal((rows, H))) * 0.5
+        self.Y = g.standard_normal((rows, D))
+        self.idx = np.sort(np.stack([g.choice(H, kc, replace=False) for _ in range(mlp_blocks)]), axis=1)
+        self.heads = max(1, min(h, attn_tiles))
+        self.tph = max(1, attn_tiles // self.heads)
+        qr = self.tph * Bt
+        self.q = g.standard_normal((self.heads, qr, d))
+        self.k = g.standard_normal((self.heads, T, d))
+        self.v = g.standard_normal((self.heads, T, d))
+        self.aidx = np.sort(np.stack([[g.choice(T, kk, replace=False) for _ in range(self.tph)]
+                                      for _ in range(self.heads)]), axis=2)
+        self.m_c = g.standard_normal((self.heads, qr))
+        self.l_c = 1.0 + g.random((self.heads, qr)) * 100
+        self.acc_c = g.standard_normal((self.heads, qr, d))
+
+    def time_step(self):
+        import oracle as O
+        w = self.w
+        t0 = time.perf_counter()
+        O.mlp_delta(self.x, self.W1, self.b1, self.W2, self.idx, self.A, self.Y, w["Bt"])
+        t1 = time.perf_counter()
+        O.attn_delta(self.q, self.k, self.v, self.aidx, self.m_c, self.l_c, self.acc_c, 1.0 / math.sqrt(w["d"]),
+                     w["Bt"])
+        t2 = time.perf_counter()
+        tiles = self.heads * self.tph
+        return ((t1 - t0) * self.nb / self.mlp_blocks + (t2 - t1) * (w["heads"] * self.nb) / tiles) * 1e6
+
+    def info(self, repeats):
+        return {"kind": "oracle", "cores": int(self.cores),
+                "sample": (f"fp64 numpy oracle: MLP delta on {self.mlp_blocks} of {self.nb} token blocks and attention "
+                           f"delta on {self.heads * self.tph} of {self.w['heads'] * self.nb} (head, query-block) "
+                           f"tiles, {repeats} run(s), extrapolated linearly to one layer-step")}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class Layer:
+    """Device-resident FLUX-shaped layer: weights, two drifted inputs, caches and selections."""
+
+    def __init__(self, w, dev, seed):
+        import torch
+        from dynamic_column_sparse_b200 import chipmunk as cm
+        self.w, self.dev, self.cm = w, dev, cm
+        T, D, H, h, d, Bt = w["T"], w["D"], w["H"], w["heads"], w["d"], w["Bt"]
+        g = torch.Generator(device=dev).manual_seed(seed)
+
+        def rn(shape, std=1.0):
+            return (torch.randn(shape, generator=g, device=dev) * std).to(torch.bfloat16)
+
+        def drift(t):
+            return (t.float() + w["sigma"] * torch.randn(t.shape, generator=g, device=dev)).to(torch.bfloat16)
+
+        self.nb = (T + Bt - 1) // Bt
+        self.kc, self.kk = k_of(H, w["mlp_permille"]), k_of(T, w["attn_permille"])
+        self.w1t, self.b1 = rn((H, D), 1 / math.sqrt(D)), rn((H,), 0.02)
+        self.w2, self.b2 = rn((H, D), 1 / math.sqrt(H)), rn((D,), 0.02)
+        x_prev = rn((T, D))
+        self.xs = [drift(x_prev)]
+        self.xs.append(drift(self.xs[0]))
+        qkv_prev = [rn((T, h, d)) for _ in range(3)]
+        self.qkvs = [[drift(t) for t in qkv_prev]]
+        self.qkvs.append([drift(t) for t in self.qkvs[0]])
+        f32, i32 = torch.float32, torch.int32
+        self.a_cache = torch.empty((self.nb, H, Bt), dtype=torch.bfloat16, device=dev)
+        self.y_cache = torch.empty((T, D), dtype=f32, device=dev)
+        self.out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+        self.idx = torch.empty((self.nb, self.kc), dtype=i32, device=dev)
+        self.mlp_scores = torch.empty((self.nb, H), dtype=f32, device=dev)
+        self.aidx = torch.empty((h, self.nb, self.kk), dtype=i32, device=dev)
+        self.m_c = torch.empty((h, T), dtype=f32, device=dev)
+        self.l_c = torch.empty((h, T), dtype=f32, device=dev)
+        self.acc_c = torch.empty((h, T, d), dtype=f32, device=dev)
+        self.o = torch.empty((T, h, d), dtype=torch.bfloat16, device=dev)
+        self.mass = torch.empty((h, self.nb, T), dtype=f32, device=dev)
+        self.ws = torch.empty(cm.mlp_workspace_bytes(T, H, self.kc, Bt), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(h * T * 4, dtype=torch.uint8, device=dev)
+        self.x_prev, self.qkv_prev = x_prev, qkv_prev
+        self.refresh()
+
+    def refresh(self, first=True):
+        cm, w = self.cm, self.w
+        cm.mlp_refresh(self.x_prev, self.w1t, self.b1, self.w2, self.b2, self.a_cache, self.y_cache, self.idx,
+                       self.mlp_scores, self.out, Bt=w["Bt"], first_step=first)
+        q, k, v = self.qkv_prev
+        cm.attn_refresh(q, k, v, self.aidx, self.m_c, self.l_c, self.acc_c, self.o, self.mass,
+                        scale=1 / math.sqrt(w["d"]), workspace=self.attn_ws)
+
+    def mlp_up(self, i):
+        self.cm.mlp_delta(self.xs[i % 2], self.w1t, self.b1, self.w2, self.idx, self.a_cache, self.y_cache, self.out,
+                          Bt=self.w["Bt"], workspace=self.ws, part="up")
+
+    def mlp_down(self, i):
+        self.cm.mlp_delta(self.xs[i % 2], self.w1t, self.b1, self.w2, self.idx, self.a_cache, self.y_cache, self.out,
+                          Bt=self.w["Bt"], workspace=self.ws, part="down")
+
+    def attn(self, i):
+        q, k, v = self.qkvs[i % 2]
+        self.cm.attn_delta(q, k, v, self.aidx, self.m_c, self.l_c, self.acc_c, self.o, scale=1 / math.sqrt(self.w["d"]))
+
+
+def time_events(fn, reps, flush, torch):
+    """Median device time (ms) of fn() over reps runs, L2 flushed before each."""
+    ts = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def source_sha(files):
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, "dynamic_column_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+KERNEL_SOURCES = {"mlp_up": ["mlp.cu", "ptx.cuh"], "mlp_down": ["mlp.cu", "ptx.cuh"], "attn_delta": ["attn.cu", "ptx.cuh"]}
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("source_sha1") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} ranks (launch with torchrun); WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    from dynamic_column_sparse_b200 import chipmunk as cm
+    cm.load_library()
+    w = dict(W)
+    L = Layer(w, dev, seed=1234 + rank)
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0, "device status set during set-up"
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    def step(i, ev=None):
+        if ev:
+            ev[0].record()
+        L.mlp_up(i)
+        if ev:
+            ev[1].record()
+        L.mlp_down(i)
+        if ev:
+            ev[2].record()
+        L.attn(i)
+        if ev:
+            ev[3].record()
+
+    for i in range(args.warmup):
+        flush()
+        step(i)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush()
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    tot = [e[0].elapsed_time(e[3]) for e in evs]
+    t_up = [e[0].elapsed_time(e[1]) for e in evs]
+    t_down = [e[1].elapsed_time(e[2]) for e in evs]
+    t_attn = [e[2].elapsed_time(e[3]) for e in evs]
+    ms_step = max_over_ranks(statistics.mean(tot))
+    status = cm.read_device_status()
+    assert status == 0, f"device status {status}"
+
+    # end to end through the public API: pinned host inputs in, outputs back, every step
+    x_h = [x.cpu().pin_memory() for x in L.xs]
+    qkv_h = [[t.cpu().pin_memory() for t in qkv] for qkv in L.qkvs]
+    out_h = torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory()
+    o_h = torch.empty(L.o.shape, dtype=L.o.dtype).pin_memory()
+    x_d = torch.empty_like(L.xs[0])
+    qkv_d = [torch.empty_like(t) for t in L.qkvs[0]]
+    w_ = L.w
+
+    def e2e_step(i):
+        x_d.copy_(x_h[i % 2], non_blocking=True)
+        for dst, src in zip(qkv_d, qkv_h[i % 2]):
+            dst.copy_(src, non_blocking=True)
+        cm.mlp_delta(x_d, L.w1t, L.b1, L.w2, L.idx, L.a_cache, L.y_cache, L.out, Bt=w_["Bt"], workspace=L.ws)
+        cm.attn_delta(*qkv_d, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, scale=1 / math.sqrt(w_["d"]))
+        out_h.copy_(L.out, non_blocking=True)
+        o_h.copy_(L.o, non_blocking=True)
+
+    for i in range(min(args.warmup, 3)):
+        e2e_step(i)
+    barrier()
+    torch.cuda.synchronize()
+    e2e_ts = []
+    for i in range(args.steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        e2e_step(i)
+        b.record()
+        b.synchronize()
+        e2e_ts.append(a.elapsed_time(b))
+    barrier()
+    e2e_ms = max_over_ranks(statistics.mean(e2e_ts))
+    h2d = x_d.numel() * 2 + sum(t.numel() * 2 for t in qkv_d)
+    d2h = out_h.numel() * 2 + o_h.numel() * 2
+
+    peaks, peak_src = load_peaks()
+    f_up, f_down, f_attn = flops_step(w)
+    flops = f_up + f_down + f_attn
+    kern = {}
+    for name, ts, fl in (("mlp_up", t_up, f_up), ("mlp_down", t_down, f_down), ("attn_delta", t_attn, f_attn)):
+        ms = statistics.mean(ts)
+        kern[name] = {"us": round(ms * 1e3, 2), "tflops": round(fl / (ms * 1e-3) / 1e12, 1),
+                      "frac_bf16_peak": round(fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    dom = max(kern, key=lambda k: kern[k]["us"])
+    dom_flops = {"mlp_up": f_up, "mlp_down": f_down, "attn_delta": f_attn}[dom]
+    achieved = dom_flops / (kern[dom]["us"] * 1e-6) / 1e12
+    tr = traffic_for(dom)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": tr, "peak_source": f"{peak_src} bf16 dense (burst)"}
+
+    us_layer = ms_step * 1e3 / world
+    res = {
+        "metric": METRIC, "value": round(us_layer, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded device Philox normals with the layer recipe's distributions (no model weights)",
+        "config": {"workload": "FLUX.1-dev 1280x768 DiT layer, sparse-delta step (MLP 70% + attention 83.5% sparse)",
+                   "T": w["T"], "d_model": w["D"], "mlp_hidden": w["H"], "heads": w["heads"], "head_dim": w["d"],
+                   "block": w["Bt"], "mlp_k": L.kc, "attn_k": L.kk, "global_batch": world, "seq_len": w["T"],
+                   "l2": "flushed before every timed step (write of a 2x L2 buffer, outside the step's events)",
+                   "parallelism": f"independent layer per GPU x{world} (no collective)"},
+        "useful_tflops": round(flops * world / (ms_step * 1e-3) / 1e12, 1),
+        "pct_bf16_peak": round(100 * flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 2),
+        "kernels": kern, "roofline": roofline,
+        "e2e": {"value": round(e2e_ms * 1e3 / world, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_rows:
+        res["rows"] = extra_rows(L, w, peaks, flush, torch, cm)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        smp = OracleSample(w)
+        us = statistics.median([smp.time_step() for _ in range(3)])
+        info = smp.info(3)
+        info["value"] = round(us, 1)
+        info["unit"] = UNIT
+        res["cpu_baseline"] = info
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    del L
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def extra_rows(L, w, peaks, flush, torch, cm):
+    """The other rows of the hot path, timed with CUDA events (median of 10, L2 flushed)."""
+    hbm = peaks["hbm_gbs"]
+    rows = {}
+    T, D, H, h, Bt = w["T"], w["D"], w["H"], w["heads"], w["Bt"]
+    reps = 10
+
+    def gbs(nbytes, ms):
+        return {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+
+    # a1: top-k over the layer's score rows, and over HunyuanVideo-length attention rows
+    ms = time_events(lambda: cm.topk_cols(L.mlp_scores, L.kc, out=L.idx), reps, flush, torch)
+    rows["topk_flux_mlp"] = dict(rows=L.nb, n=H, k=L.kc, **gbs(L.nb * (H + L.kc) * 4, ms))
+    mass2 = L.mass.view(h * L.nb, T)
+    aidx2 = L.aidx.view(h * L.nb, L.kk)
+    ms = time_events(lambda: cm.topk_cols(mass2, L.kk, out=aidx2), reps, flush, torch)
+    rows["topk_flux_attn"] = dict(rows=h * L.nb, n=T, k=L.kk, **gbs(h * L.nb * (T + L.kk) * 4, ms))
+    g = torch.Generator(device=L.dev).manual_seed(7)
+    hn, hk, hr = 118800, 8316, 148 * 20
+    hs = torch.rand((hr, hn), generator=g, device=L.dev) ** 4
+    hidx = torch.empty((hr, hk), dtype=torch.int32, device=L.dev)
+    ms = time_events(lambda: cm.topk_cols(hs, hk, out=hidx), 3, flush, torch)
+    rows["topk_hunyuan_attn_rows"] = dict(rows=hr, n=hn, k=hk, note="2960 of 22296 HunyuanVideo mass rows",
+                                          **gbs(hr * (hn + hk) * 4, ms))
+    del hs, hidx
+    # a6: cache column gather / scatter (FLUX and HunyuanVideo-sized caches)
+    packed = torch.empty((L.nb, L.kc, Bt), dtype=torch.bfloat16, device=L.dev)
+    nbytes = 2 * L.nb * L.kc * Bt * 2
+    ms = time_events(lambda: cm.gather_cols(L.a_cache, L.idx, packed), reps, flush, torch)
+    rows["gather_flux"] = gbs(nbytes, ms)
+    ms = time_events(lambda: cm.scatter_cols(packed, L.idx, L.a_cache), reps, flush, torch)
+    rows["scatter_flux"] = gbs(nbytes, ms)
+    del packed
+    nbh = (118800 + 127) // 128
+    cache_h = torch.zeros((nbh, H, Bt), dtype=torch.bfloat16, device=L.dev)
+    idx_h = torch.sort(torch.rand((nbh, H), generator=g, device=L.dev).argsort(dim=1)[:, :L.kc], dim=1)[0]
+    idx_h = idx_h.to(torch.int32).contiguous()
+    packed_h = torch.empty((nbh, L.kc, Bt), dtype=torch.bfloat16, device=L.dev)
+    nbytes = 2 * nbh * L.kc * Bt * 2
+    ms = time_events(lambda: cm.gather_cols(cache_h, idx_h, packed_h), 5, flush, torch)
+    rows["gather_hunyuan"] = gbs(nbytes, ms)
+    ms = time_events(lambda: cm.scatter_cols(packed_h, idx_h, cache_h), 5, flush, torch)
+    rows["scatter_hunyuan"] = gbs(nbytes, ms)
+    del cache_h, idx_h, packed_h
+    # a5: dense refresh of the layer
+    ms_mlp = time_events(lambda: cm.mlp_refresh(L.x_prev, L.w1t, L.b1, L.w2, L.b2, L.a_cache, L.y_cache, L.idx,
+                                                L.mlp_scores, L.out, Bt=Bt), 5, flush, torch)
+    q, k, v = L.qkv_prev
+    ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, L.mass,
+                                                  scale=1 / math.sqrt(w["d"]), workspace=L.attn_ws), 5, flush, torch)
+    dense_mlp_f = 4 * T * D * H
+    dense_attn_f = 4 * T * T * w["d"] * h
+    rows["refresh_mlp"] = {"us": round(ms_mlp * 1e3, 1),
+                           "tflops": round(dense_mlp_f / (ms_mlp * 1e-3) / 1e12, 1)}
+    rows["refresh_attn"] = {"us": round(ms_attn * 1e3, 1), "passes": "dense + mass + top-k + complement",
+                            "tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1)}
+    # dense layer at the same shape with the same kernels (k = all columns, all keys)
+    idx_all = torch.arange(H, dtype=torch.int32, device=L.dev).repeat(L.nb, 1).contiguous()
+    ws_all = torch.empty(cm.mlp_workspace_bytes(T, H, H, Bt), dtype=torch.uint8, device=L.dev)
+    aidx_all = torch.arange(T, dtype=torch.int32, device=L.dev).repeat(h, L.nb, 1).contiguous()
+    m0 = torch.full((h, T), float("-inf"), device=L.dev)
+    l0 = torch.zeros((h, T), device=L.dev)
+    a0 = torch.zeros((h, T, w["d"]), device=L.dev)
+    ms_dm = time_events(lambda: cm.mlp_delta(L.xs[0], L.w1t, L.b1, L.w2, idx_all, L.a_cache, L.y_cache, L.out,
+                                             Bt=Bt, workspace=ws_all), 5, flush, torch)
+    ms_da = time_events(lambda: cm.attn_delta(q, k, v, aidx_all, m0, l0, a0, L.o, scale=1 / math.sqrt(w["d"])), 5,
+                        flush, torch)
+    rows["dense_layer_k_all"] = {"us": round((ms_dm + ms_da) * 1e3, 1), "mlp_us": round(ms_dm * 1e3, 1),
+                                 "attn_us": round(ms_da * 1e3, 1),
+                                 "tflops": round((dense_mlp_f + dense_attn_f) / ((ms_dm + ms_da) * 1e-3) / 1e12, 1)}
+    xw = L.xs[0]
+    w1 = L.w1t.t()
+    ms_cub = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),
+                                              L.w2), 5, flush, torch)
+    rows["dense_mlp_torch_context"] = {"us": round(ms_cub * 1e3, 1), "note": "torch.matmul (cuBLAS) + GELU, context only"}
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    return rows
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = dict(W)
+    smp = OracleSample(w, mlp_blocks=2, attn_tiles=24)
+    for _ in range(args.warmup):
+        smp.time_step()
+    vals = [smp.time_step() for _ in range(args.steps)]
+    us = statistics.mean(vals)
+    info = smp.info(args.steps)
+    info["value"] = round(us, 1)
+    info["unit"] = UNIT
+    res = {"impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3), "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic: seeded numpy normals with the layer recipe's shapes",
+           "config": {"workload": "FLUX.1-dev 1280x768 DiT layer, sparse-delta step (MLP 70% + attention 83.5% sparse)",
+                      "T": w["T"], "d_model": w["D"], "mlp_hidden": w["H"], "heads": w["heads"],
+                      "head_dim": w["d"], "block": w["Bt"]},
+           "cpu_baseline": info,
+           "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the extra hot-path rows")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

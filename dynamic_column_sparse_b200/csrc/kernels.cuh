@@ -1,0 +1,91 @@
+// kernels.cuh - parameter blocks and host launchers of the library's kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cm {
+
+// ------------------------------------------------------------------ top-k
+
+struct TopkParams {
+  const float *scores;
+  int64_t rows, n, ld_scores;
+  int32_t k;
+  int32_t *idx;
+  int64_t ld_idx;
+};
+cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
+
+// ------------------------------------------------------------------ cache column gather / scatter
+
+cudaError_t launch_gather_cols(const uint16_t *a_cache, int64_t nb, int64_t H, int Bt, const int32_t *idx, int k,
+                               uint16_t *packed, cudaStream_t s);
+cudaError_t launch_scatter_cols(const uint16_t *packed, int64_t nb, int64_t H, int Bt, const int32_t *idx, int k,
+                                uint16_t *a_cache, cudaStream_t s);
+
+// ------------------------------------------------------------------ MLP
+
+enum MlpUpMode : int { kUpDelta = 0, kUpRefresh = 1, kUpRefreshFirst = 2 };
+
+// Kernel 1: a = gelu(x W1[:, S] + b1[S]) over gathered hidden columns, with
+// the delta / cache-writeback (sparse step) or score / cache-rebuild (refresh)
+// epilogue. One CTA per (token block, chunk of 128 selected columns).
+struct MlpUpParams {
+  int T, D, H, k, Bt, nb, nchunks, k_pad, mode;
+  const int32_t *idx;     // [nb][k] (sparse step)
+  const uint16_t *b1;     // [H]
+  uint16_t *a_cache;      // [nb][H][Bt]
+  uint16_t *delta;        // [nb][k_pad][Bt] (sparse step)
+  float *scores;          // [nb][H] (refresh)
+  int *status;
+};
+cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t_gather, const CUtensorMap &tm_x,
+                          cudaStream_t s);
+
+enum MlpDownMode : int { kDownAccumulate = 0, kDownOverwrite = 1 };
+
+// Kernel 2: Y[b, n-slice] (+)= A[b] W2[S_b, n-slice] where A is the delta
+// workspace (sparse step, rows gathered from W2) or the rebuilt activation
+// cache (refresh, all rows). One CTA per (token block, slice of BN columns).
+struct MlpDownParams {
+  int T, D, Bt, nb, krows, k, n_slices, bn, mode;
+  const int32_t *idx;     // [nb][k] (sparse step)
+  const uint16_t *b2;     // [D] (refresh)
+  float *y_cache;         // [T][D]
+  uint16_t *out;          // [T][D] or nullptr
+  int *status;
+};
+// tm_a: 3-D map over A [nb][rows][Bt]; tm_w2: gather4 map (sparse) or tile map (dense) over W2 [H][D].
+cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
+                            cudaStream_t s);
+
+// ------------------------------------------------------------------ attention
+
+enum AttnMode : int { kAttnDelta = 0, kAttnDense = 1, kAttnComplement = 2 };
+
+struct AttnParams {
+  int T, h, nb, k;
+  float scale_log2;       // logit scale * log2(e)
+  const int32_t *idx;     // [h][nb][k]
+  float *m_c, *l_c, *acc_c;  // [h][T], [h][T], [h][T][128]
+  uint16_t *o;            // [T][h][128]
+  float *lse;             // [h][T] (dense)
+  int *status;
+};
+// tm_q: tile map over Q [T][h*128] (box 64 x 128). tm_k / tm_v: gather4 maps
+// (sparse step) or tile maps (dense, complement) over K, V [T][h*128].
+cudaError_t launch_attn(int mode, const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                        const CUtensorMap &tm_v, cudaStream_t s);
+
+struct MassParams {
+  int T, h, nb;
+  float scale_log2;
+  const float *lse;       // [h][T]
+  float *mass;            // [h][nb][T]
+  int *status;
+};
+cudaError_t launch_attn_mass(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k, cudaStream_t s);
+
+}  // namespace cm

@@ -1,0 +1,448 @@
+// mlp.cu - gathered-column MLP kernels of the sparse delta step and the refresh.
+//
+// Kernel 1 (mlp_up): one CTA per (token block b, chunk of 128 selected hidden
+// columns). The selected rows of W1^T are gathered from global memory into
+// 128-byte-swizzled shared-memory tiles with TMA gather4 (four arbitrary rows
+// per instruction), the token block of x arrives by a tiled TMA load, and one
+// thread issues tcgen05 bf16 MMAs accumulating D[col][token] in TMEM. The
+// epilogue warps own one hidden column each (one TMEM lane) and all Bt tokens
+// of it, so the activation cache run a_cache[b][c][0..Bt) and the delta row
+// are read and written as whole contiguous runs.
+//
+// Kernel 2 (mlp_down): one CTA per (token block b, slice of BN model columns).
+// The K dimension runs over the selected hidden units: the delta rows come
+// from the workspace by tiled TMA, the matching W2 rows are gathered with TMA
+// gather4; both operands are MN-major. The epilogue adds the fp32 result into
+// the output cache (or overwrites it with result + b2 on a refresh) and writes
+// the bf16 layer output.
+//
+// Warp roles in both kernels: warp 0 = TMA producer, warp 1 = MMA issuer
+// (and TMEM owner), warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
+#include <algorithm>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace cm {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBK = 64;  // K elements per pipeline stage = one 128-byte swizzle row
+
+// Warp-uniform bounded wait: every lane polls, the warp leaves together.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
+  const bool ok = mbar_wait(bar, parity, status, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int BT>
+struct UpCfg {
+  static constexpr int kStages = BT == 128 ? 3 : 4;
+  static constexpr uint32_t kABytes = 128 * 128;  // 128 gathered rows x 64 bf16
+  static constexpr uint32_t kBBytes = BT * 128;   // BT tokens x 64 bf16
+  static constexpr uint32_t kBarOff = kStages * (kABytes + kBBytes);
+  static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
+};
+
+template <int BT>
+__global__ void __launch_bounds__(kThreads, 1)
+    mlp_up_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
+                  const MlpUpParams p) {
+  using C = UpCfg<BT>;
+  constexpr uint32_t kIdesc = idesc_bf16(128, BT, false, false);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align_up<1024>(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + C::kStages * C::kABytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+  uint64_t *empty = full + C::kStages;
+  uint64_t *acc_full = empty + C::kStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *rows = reinterpret_cast<int *>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*(volatile int *)p.status != kDevOk) return;
+  const int chunk = blockIdx.x % p.nchunks;
+  const int b = blockIdx.x / p.nchunks;
+  const bool sparse = p.mode == kUpDelta;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w1t);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BT);
+    tmem_relinquish();
+  }
+  if (threadIdx.x < 128) {
+    const int j = chunk * 128 + threadIdx.x;
+    int c;
+    if (sparse) {
+      c = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
+      if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the cache
+        atomicCAS(p.status, kDevOk, kDevBadIndex);
+        c = 0;
+      }
+    } else {
+      c = min(j, p.H - 1);
+    }
+    rows[threadIdx.x] = c;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = p.D / kBK;
+
+  if (warp == 0) {
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::kStages;
+      const uint32_t ph = (kb / C::kStages) & 1;
+      if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::kABytes + C::kBBytes);
+      __syncwarp();
+      tma_gather4(sA + s * C::kABytes + lane * 512, &tm_w1t, &full[s], kb * kBK, rows[4 * lane], rows[4 * lane + 1],
+                  rows[4 * lane + 2], rows[4 * lane + 3]);
+      if (lane == 0) tma_load_2d(sB + s * C::kBBytes, &tm_x, &full[s], kb * kBK, b * BT);
+    }
+  } else if (warp == 1) {
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::kStages;
+      const uint32_t ph = (kb / C::kStages) & 1;
+      if (!wait_warp(&full[s], ph, p.status, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a0 = smem_u32(sA + s * C::kABytes);
+        const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+          umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (ok && lane == 0) umma_commit(acc_full);
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    if (wait_warp(acc_full, 0, p.status, abort_flag)) {
+      tc_fence_after();
+      const int j = chunk * 128 + r;
+      const bool valid_j = sparse ? (j < p.k) : (j < p.H);
+      const int c = rows[r];
+      const int nvalid = min(BT, p.T - b * BT);
+      const float bias = bf16_bits_to_f32(__ldg(p.b1 + c));
+      uint16_t *arow = p.a_cache + (static_cast<size_t>(b) * p.H + c) * BT;
+      uint16_t *drow = sparse ? p.delta + (static_cast<size_t>(b) * p.k_pad + j) * BT : nullptr;
+      const bool first = p.mode == kUpRefreshFirst;
+      float score = 0.f;
+#pragma unroll 1
+      for (int tq = 0; tq < BT / 32; ++tq) {
+        float acc[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + tq * 32, acc);
+        uint4 oldv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                         make_uint4(0, 0, 0, 0)};
+        if (valid_j) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(arow + tq * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) oldv[v] = src[v];
+        }
+        const uint16_t *old = reinterpret_cast<const uint16_t *>(oldv);
+        uint32_t na[16], dl[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          uint16_t nab[2], dlb[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = tq * 32 + i + u;
+            const float a = gelu_tanh(acc[i + u] + bias);
+            const uint16_t abf = f32_to_bf16_bits(a);
+            const bool tok = t < nvalid;
+            const float o = bf16_bits_to_f32(old[i + u]);
+            nab[u] = tok ? abf : old[i + u];
+            if (sparse) {
+              dlb[u] = (valid_j && tok) ? f32_to_bf16_bits(bf16_bits_to_f32(abf) - o) : static_cast<uint16_t>(0);
+            } else {
+              dlb[u] = 0;
+              score += tok ? fabsf(first ? a : a - o) : 0.f;
+            }
+          }
+          na[i / 2] = static_cast<uint32_t>(nab[0]) | (static_cast<uint32_t>(nab[1]) << 16);
+          dl[i / 2] = static_cast<uint32_t>(dlb[0]) | (static_cast<uint32_t>(dlb[1]) << 16);
+        }
+        if (valid_j) {
+          uint4 *dst = reinterpret_cast<uint4 *>(arow + tq * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(na[4 * v], na[4 * v + 1], na[4 * v + 2], na[4 * v + 3]);
+        }
+        if (sparse) {
+          uint4 *dst = reinterpret_cast<uint4 *>(drow + tq * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(dl[4 * v], dl[4 * v + 1], dl[4 * v + 2], dl[4 * v + 3]);
+        }
+      }
+      if (!sparse && valid_j) p.scores[static_cast<size_t>(b) * p.H + c] = score;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, BT);
+}
+
+template <int BN>
+struct DownCfg {
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kABytes = 128 * 128;         // 64 K-rows x 128 tokens (two 64-token atoms)
+  static constexpr uint32_t kBBytes = (BN / 64) * 8192;  // 64 K-rows x BN columns
+  static constexpr uint32_t kBarOff = kStages * (kABytes + kBBytes);
+  static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
+};
+
+template <int BT, int BN, bool DENSE>
+__global__ void __launch_bounds__(kThreads, 1)
+    mlp_down_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w2,
+                    const MlpDownParams p) {
+  using C = DownCfg<BN>;
+  constexpr uint32_t kIdesc = idesc_bf16(128, BN, true, true);
+  constexpr uint32_t kTx = (BT / 64) * 8192 + C::kBBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align_up<1024>(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + C::kStages * C::kABytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+  uint64_t *empty = full + C::kStages;
+  uint64_t *acc_full = empty + C::kStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*(volatile int *)p.status != kDevOk) return;
+  const int slice = blockIdx.x % p.n_slices;
+  const int b = blockIdx.x / p.n_slices;
+  const int n0 = slice * BN;
+  const int kext = DENSE ? p.krows : p.k;
+  const int nk = (kext + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_w2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  if (BT == 64) {
+    // tokens 64..127 of every A stage stay zero: the MMA always runs M = 128
+    for (int s = 0; s < C::kStages; ++s) {
+      uint4 *z = reinterpret_cast<uint4 *>(sA + s * C::kABytes + 8192);
+      for (int i = threadIdx.x; i < 8192 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    fence_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    const int32_t *irow = DENSE ? nullptr : p.idx + static_cast<size_t>(b) * p.k;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::kStages;
+      const uint32_t ph = (kb / C::kStages) & 1;
+      if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], kTx);
+#pragma unroll
+        for (int mt = 0; mt < BT / 64; ++mt)
+          tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &full[s], mt * 64, kb * kBK, b);
+        if (DENSE) {
+#pragma unroll
+          for (int ns = 0; ns < BN / 64; ++ns)
+            tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &full[s], n0 + ns * 64, kb * kBK);
+        }
+      }
+      __syncwarp();
+      if (!DENSE) {
+        // 16 groups of 4 rows per 64-column slab; lane l issues groups l, l+32, ...
+        for (int g = lane; g < 16 * (BN / 64); g += 32) {
+          const int ns = g >> 4, grp = g & 15;
+          const int j0 = kb * kBK + grp * 4;
+          int c[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[e] = __ldg(irow + min(j0 + e, p.k - 1));
+          tma_gather4(sB + s * C::kBBytes + ns * 8192 + grp * 512, &tm_w2, &full[s], n0 + ns * 64, c[0], c[1], c[2],
+                      c[3]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::kStages;
+      const uint32_t ph = (kb / C::kStages) & 1;
+      if (!wait_warp(&full[s], ph, p.status, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a0 = smem_u32(sA + s * C::kABytes);
+        const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 8192, 1024);
+          const uint64_t bd = sdesc_sw128(b0 + kk * 2048, 8192, 1024);
+          umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (ok && lane == 0) umma_commit(acc_full);
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int t = q * 32 + lane;
+    const int64_t grow = static_cast<int64_t>(b) * BT + t;
+    const bool valid = t < BT && grow < p.T;
+    if (wait_warp(acc_full, 0, p.status, abort_flag)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int nc = 0; nc < BN / 32; ++nc) {
+        float acc[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + nc * 32, acc);
+        if (valid) {
+          const int n = n0 + nc * 32;
+          float4 *y4 = reinterpret_cast<float4 *>(p.y_cache + grow * p.D + n);
+          float y[32];
+          if (p.mode == kDownAccumulate) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 o = y4[v];
+              y[4 * v] = o.x + acc[4 * v];
+              y[4 * v + 1] = o.y + acc[4 * v + 1];
+              y[4 * v + 2] = o.z + acc[4 * v + 2];
+              y[4 * v + 3] = o.w + acc[4 * v + 3];
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[i] = acc[i] + bf16_bits_to_f32(__ldg(p.b2 + n + i));
+          }
+#pragma unroll
+          for (int v = 0; v < 8; ++v) y4[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+          if (p.out != nullptr) {
+            uint4 *o4 = reinterpret_cast<uint4 *>(p.out + grow * p.D + n);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              o4[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]), pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
+                                 pack_bf16x2(y[8 * v + 4], y[8 * v + 5]), pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, BN);
+}
+
+// out = bf16(y) when a sparse step selects nothing
+__global__ void y_to_out_kernel(const float4 *__restrict__ y, uint2 *__restrict__ out, int64_t n4) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = y[i];
+    out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, uint32_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+template <int BT>
+cudaError_t launch_up_t(const MlpUpParams &p, const CUtensorMap &w, const CUtensorMap &x, cudaStream_t s) {
+  using C = UpCfg<BT>;
+  cudaError_t e = set_smem(mlp_up_kernel<BT>, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = static_cast<int64_t>(p.nb) * p.nchunks;
+  mlp_up_kernel<BT><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(w, x, p);
+  return cudaGetLastError();
+}
+
+template <int BT, int BN, bool DENSE>
+cudaError_t launch_down_t(const MlpDownParams &p, const CUtensorMap &a, const CUtensorMap &w, cudaStream_t s) {
+  using C = DownCfg<BN>;
+  cudaError_t e = set_smem(mlp_down_kernel<BT, BN, DENSE>, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = static_cast<int64_t>(p.nb) * p.n_slices;
+  mlp_down_kernel<BT, BN, DENSE><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(a, w, p);
+  return cudaGetLastError();
+}
+
+template <int BT, bool DENSE>
+cudaError_t launch_down_bn(const MlpDownParams &p, const CUtensorMap &a, const CUtensorMap &w, cudaStream_t s) {
+  switch (p.bn) {
+    case 256: return launch_down_t<BT, 256, DENSE>(p, a, w, s);
+    case 128: return launch_down_t<BT, 128, DENSE>(p, a, w, s);
+    case 64: return launch_down_t<BT, 64, DENSE>(p, a, w, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t_gather, const CUtensorMap &tm_x,
+                          cudaStream_t s) {
+  if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
+  if (p.Bt == 128) return launch_up_t<128>(p, tm_w1t_gather, tm_x, s);
+  if (p.Bt == 64) return launch_up_t<64>(p, tm_w1t_gather, tm_x, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
+                            cudaStream_t s) {
+  if (p.nb <= 0) return cudaSuccess;
+  const int kext = dense ? p.krows : p.k;
+  if (kext <= 0) {
+    if (p.out == nullptr) return cudaSuccess;
+    const int64_t n4 = static_cast<int64_t>(p.T) * p.D / 4;
+    y_to_out_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 16)), 256, 0, s>>>(
+        reinterpret_cast<const float4 *>(p.y_cache), reinterpret_cast<uint2 *>(p.out), n4);
+    return cudaGetLastError();
+  }
+  if (p.Bt == 128) return dense ? launch_down_bn<128, true>(p, tm_a, tm_w2, s) : launch_down_bn<128, false>(p, tm_a, tm_w2, s);
+  if (p.Bt == 64) return dense ? launch_down_bn<64, true>(p, tm_a, tm_w2, s) : launch_down_bn<64, false>(p, tm_a, tm_w2, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cm

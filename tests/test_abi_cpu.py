@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/chipmunk.h declares, and rejects bad arguments
+before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "chipmunk.h")
+
+
+@pytest.fixture(scope="module")
+def cm():
+    import torch  # noqa: F401  (loads the CUDA runtime the library links against)
+    from dynamic_column_sparse_b200 import build, chipmunk
+    build.build()
+    return chipmunk
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:[A-Za-z_][\w \*]*?)\b(chipmunk_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("chipmunk_topk_cols", "chipmunk_mlp_delta", "chipmunk_attn_delta", "chipmunk_dense_refresh"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(cm):
+    lib = cm.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(cm.EXPORTS) <= set(declared_functions())
+
+
+def test_struct_layouts_match_the_header(cm):
+    # int64 x3 + int32 x2 + 9 pointers
+    assert ctypes.sizeof(cm.MlpArgs) == 24 + 8 + 9 * 8
+    # int64 + int32 x4 + float + pad + 8 pointers
+    assert ctypes.sizeof(cm.AttnArgs) == 8 + 16 + 4 + 4 + 8 * 8
+    assert cm.RefreshArgs.mlp.offset == 8
+    assert cm.RefreshArgs.scores.offset == 8 + ctypes.sizeof(cm.MlpArgs) + ctypes.sizeof(cm.AttnArgs)
+
+
+def test_version_and_status_strings(cm):
+    lib = cm.load_library()
+    assert cm.version() == "0.1.0"
+    for st in range(8):
+        assert lib.chipmunk_status_string(st)
+    assert b"unknown" in lib.chipmunk_status_string(99)
+
+
+def _mlp_args(cm, **kw):
+    base = dict(T=256, D=128, H=512, Bt=64, k=128, x=0x1000, w1t=0x2000, b1=0x3000, w2=0x4000, b2=0x5000,
+                idx=0x6000, a_cache=0x7000, y_cache=0x8000, out=0)
+    base.update(kw)
+    return cm.MlpArgs(**base)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("D", 100, 2), ("D", 0, 2), ("Bt", 32, 2), ("k", 513, 1), ("k", -1, 1), ("T", 0, 2),
+    ("x", 0, 1), ("w1t", 0x2008, 3), ("y_cache", 0, 1),
+])
+def test_mlp_delta_rejects_bad_arguments_on_the_host(cm, field, value, status):
+    lib = cm.load_library()
+    a = _mlp_args(cm, **{field: value})
+    st = lib.chipmunk_mlp_delta(ctypes.byref(a), None, 0, None)
+    assert st == status, lib.chipmunk_last_error()
+    assert lib.chipmunk_last_error()
+
+
+def test_mlp_delta_requires_workspace(cm):
+    lib = cm.load_library()
+    a = _mlp_args(cm)
+    need = lib.chipmunk_workspace_bytes(cm.OP_MLP_DELTA, ctypes.byref(a))
+    assert need == 4 * 128 * 64 * 2  # nb * round_up(k,128) * Bt bf16
+    st = lib.chipmunk_mlp_delta(ctypes.byref(a), None, 0, None)
+    assert st == 7
+
+
+@pytest.mark.parametrize("field,value,status", [("d", 64, 2), ("Bt", 64, 2), ("k", 301, 1), ("h", 0, 2), ("q", 0, 1)])
+def test_attn_delta_rejects_bad_arguments_on_the_host(cm, field, value, status):
+    lib = cm.load_library()
+    base = dict(T=300, h=2, d=128, Bt=128, k=40, scale=0.088, q=0x1000, kk=0x2000, v=0x3000, idx=0x4000,
+                m_c=0x5000, l_c=0x6000, acc_c=0x7000, o=0x8000)
+    base[field] = value
+    a = cm.AttnArgs(**base)
+    assert lib.chipmunk_attn_delta(ctypes.byref(a), None, 0, None) == status
+
+
+def test_topk_rejects_bad_arguments_on_the_host(cm):
+    lib = cm.load_library()
+    assert lib.chipmunk_topk_cols(ctypes.c_void_p(0x1000), 4, 10, 10, 11, ctypes.c_void_p(0x2000), 11, None, 0, None) == 1
+    assert lib.chipmunk_topk_cols(ctypes.c_void_p(0x1000), 4, 10, 9, 3, ctypes.c_void_p(0x2000), 3, None, 0, None) == 2
+    assert lib.chipmunk_topk_cols(ctypes.c_void_p(0x1004), 4, 10, 10, 3, ctypes.c_void_p(0x2000), 3, None, 0, None) == 3
+    # nothing to do is not an error
+    assert lib.chipmunk_topk_cols(None, 0, 10, 10, 3, None, 3, None, 0, None) == 0
+    assert lib.chipmunk_topk_cols(None, 4, 10, 10, 0, None, 0, None, 0, None) == 0
+
+
+def test_refresh_rejects_unknown_kind(cm):
+    lib = cm.load_library()
+    r = cm.RefreshArgs(kind=7, scores=0x1000)
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1
+    r = cm.RefreshArgs(kind=cm.REFRESH_ATTN, scores=0)
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1

@@ -1,0 +1,56 @@
+"""Top-k column selection on the GPU against the oracle: bit-exact indices on
+the same fp32 score rows (ties to the lower index)."""
+import numpy as np
+import pytest
+
+import oracle as O
+from dynamic_column_sparse_b200 import synth
+from helpers import dev_f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cm():
+    from dynamic_column_sparse_b200 import chipmunk
+    chipmunk.load_library()
+    return chipmunk
+
+
+@pytest.mark.parametrize("rows,n,k,ties", [
+    (4, 512, 128, False),        # tiny MLP: 4 blocks x 512 hidden, 25%
+    (4, 512, 128, True),
+    (34, 12288, 3686, True),     # FLUX MLP scores
+    (816, 4352, 718, True),      # FLUX attention mass rows (24 heads x 34 blocks)
+    (7, 40960, 4096, True),      # longest row staged in shared memory
+    (7, 40961, 4096, True),      # shortest row read from global memory
+    (300, 118800, 8316, True),   # HunyuanVideo attention row length, two waves of the grid
+    (3, 1000, 1, False),
+    (3, 1000, 999, True),
+])
+def test_topk_matches_oracle(cm, rows, n, k, ties):
+    s = synth.score_rows(7, rows, n, ties=ties)
+    got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
+    np.testing.assert_array_equal(got, O.topk_cols(s, k))
+
+
+def test_topk_special_values(cm):
+    n = 3000
+    rows = []
+    rows.append(np.full(n, 0.5, dtype=np.float32))                       # all equal
+    r = np.zeros(n, dtype=np.float32); r[::2] = -0.0; rows.append(r)      # -0 ties +0
+    r = synth.score_rows(3, 1, n)[0] - 1.0; rows.append(r)                # negatives
+    r = synth.score_rows(4, 1, n)[0]; r[[5, 17, 2999]] = np.inf; r[[7, 8]] = -np.inf; rows.append(r)
+    r = np.round(synth.score_rows(5, 1, n)[0] * 2) / 2; rows.append(r.astype(np.float32))  # few distinct values
+    s = np.stack(rows).astype(np.float32)
+    for k in (0, 1, 2, 100, 1500, 2999, 3000):
+        got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
+        np.testing.assert_array_equal(got, O.topk_cols(s, k), err_msg=f"k={k}")
+
+
+def test_topk_tiny_rows(cm):
+    for n in (1, 2, 3, 31, 33):
+        s = synth.score_rows(n, 5, n, ties=True)
+        for k in range(0, n + 1, max(1, n // 3)):
+            got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
+            np.testing.assert_array_equal(got, O.topk_cols(s, k))
