@@ -35,8 +35,9 @@ EXPORTS = (
     "chipmunk_topk_cols", "chipmunk_mlp_delta", "chipmunk_mlp_delta_up", "chipmunk_mlp_delta_down",
     "chipmunk_attn_delta", "chipmunk_dense_refresh",
     "chipmunk_gather_cols", "chipmunk_scatter_cols", "chipmunk_workspace_bytes", "chipmunk_status_string",
-    "chipmunk_last_error", "chipmunk_read_device_status", "chipmunk_version",
+    "chipmunk_last_error", "chipmunk_read_device_status", "chipmunk_version", "chipmunk_mlp_delta_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class ChipmunkError(RuntimeError):
@@ -96,6 +97,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "chipmunk_gather_cols": [vp, i64, i64, i32, vp, i32, vp, vp],
             "chipmunk_scatter_cols": [vp, i64, i64, i32, vp, i32, vp, vp],
             "chipmunk_read_device_status": [ctypes.POINTER(i32), vp],
+            "chipmunk_mlp_delta_noalloc": [ctypes.POINTER(MlpArgs), vp],
         }
         for name, argtypes in sig.items():
             fn = getattr(lib, name)
@@ -220,6 +222,16 @@ def mlp_delta(x, w1t, b1, w2, idx, a_cache, y_cache, out=None, Bt=128, workspace
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     fn = {None: lib.chipmunk_mlp_delta, "up": lib.chipmunk_mlp_delta_up, "down": lib.chipmunk_mlp_delta_down}[part]
     _check(fn(ctypes.byref(a), _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+def mlp_delta_noalloc(x, w1t, b1, w2, idx, a_cache, y_cache, out=None, Bt=128, stream=None):
+    """mlp_delta without caller scratch: for callers that cannot allocate device
+    memory. The library's fixed 64 MiB scratch array is shared by every call, so
+    calls must not overlap on the GPU; larger problems raise."""
+    lib = load_library()
+    a = _mlp_args(x, w1t, b1, w2, None, idx, a_cache, y_cache, out, Bt, idx.shape[1])
+    _check(lib.chipmunk_mlp_delta_noalloc(ctypes.byref(a), _stream(stream)))
     return out
 
 

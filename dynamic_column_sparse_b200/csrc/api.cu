@@ -408,6 +408,50 @@ chipmunk_status chipmunk_scatter_cols(const void *packed, int64_t nb, int64_t H,
   return CHIPMUNK_OK;
 }
 
+// Scratch of chipmunk_mlp_delta_noalloc: a fixed device array, one per device,
+// so that callers without an allocator can run the sparse MLP step. In host
+// code this name is a host-side stand-in; its device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CHIPMUNK_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[kMaxDevices] = {};
+
+// One-time per-device look-up of the scratch array's device address, with
+// that device current (the caller's current device).
+static chipmunk_status noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(CHIPMUNK_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CHIPMUNK_OK;
+}
+
+chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args *a, chipmunk_stream stream) {
+  CM_CHECK(check_mlp(a, false));
+  const size_t need = mlp_delta_ws(a);
+  if (need > CHIPMUNK_NOALLOC_SCRATCH_BYTES)
+    return fail(CHIPMUNK_ERR_WORKSPACE,
+                "chipmunk_mlp_delta_noalloc needs %zu bytes of scratch, more than its fixed %zu; "
+                "use chipmunk_mlp_delta with a caller workspace",
+                need, size_t(CHIPMUNK_NOALLOC_SCRATCH_BYTES));
+  int *status = nullptr;
+  CM_CHECK(device_setup(&status));
+  void *ws = nullptr;
+  CM_CHECK(noalloc_scratch(&ws));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CM_CHECK(mlp_up_impl(a, ws, status, s));
+  return mlp_down_impl(a, ws, status, s);
+}
+
 chipmunk_status chipmunk_read_device_status(int32_t *host_out, chipmunk_stream stream) {
   if (host_out == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "host_out is NULL");
   int *status = nullptr;

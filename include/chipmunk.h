@@ -197,6 +197,34 @@ CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_down(const chipmunk_mlp_args *a,
                                         chipmunk_stream stream);
 
 /*
+ * chipmunk_mlp_delta_noalloc - the sparse MLP step for callers that cannot
+ * allocate device memory. No counterpart in the paper: the post describes the
+ * method, not how its scratch memory is obtained.
+ *
+ * Some callers can't call cudaMalloc: a host framework that owns all device
+ * memory and gives its plugins no allocator, or a latency-bound loop where an
+ * allocation would synchronise the device. This call computes exactly what
+ * chipmunk_mlp_delta computes, with the same arguments, but takes its delta
+ * scratch from a fixed array inside the library instead of from the caller:
+ *   - The array holds CHIPMUNK_NOALLOC_SCRATCH_BYTES (64 MiB). Every GPU that
+ *     loads the library keeps it until the process exits.
+ *   - Calls that need more (nb * round_up(k, 128) * Bt * 2 bytes; the
+ *     FLUX.1-dev layer at 70% sparsity needs 32.3 MB) return
+ *     CHIPMUNK_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up per device, done with that device current); make that
+ *     first call before any stream capture.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each call writes every scratch
+ *     byte it reads before reading it), but calls whose work overlaps on the
+ *     GPU (different streams, or different host threads without ordering)
+ *     race on it and must be serialised by the caller.
+ */
+#define CHIPMUNK_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args *a, chipmunk_stream stream);
+
+/*
  * Sparse attention step (post: attention output as a sum of scaled rows of V,
  * of which only a subset is replaced each step). For each head and 128-query
  * block the selected keys idx[h][b] are attended with the current q, kk, v by
