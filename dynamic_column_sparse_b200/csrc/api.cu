@@ -201,10 +201,11 @@ chipmunk_status mlp_up_impl(const chipmunk_mlp_args *a, void *ws, int *status, c
   const int64_t nb = ceil_div(a->T, a->Bt);
   const int64_t nchunks = ceil_div(a->k, 128);
   CUtensorMap tm_w1t, tm_x;
-  CM_CHECK(map2d(&tm_w1t, a->w1t, a->H, a->D, 64, 1, "w1t gather"));
+  CM_CHECK(map2d(&tm_w1t, a->w1t, a->H, a->D, 64, 128, "w1t"));
   CM_CHECK(map2d(&tm_x, a->x, a->T, a->D, 64, a->Bt, "x"));
   cm::MlpUpParams up{int(a->T), int(a->D), int(a->H), a->k, a->Bt, int(nb), int(nchunks), int(nchunks * 128),
-                     cm::kUpDelta, a->idx, static_cast<const uint16_t *>(a->b1), static_cast<uint16_t *>(a->a_cache),
+                     cm::kUpDelta, static_cast<const uint16_t *>(a->w1t), a->idx,
+                     static_cast<const uint16_t *>(a->b1), static_cast<uint16_t *>(a->a_cache),
                      static_cast<uint16_t *>(ws), nullptr, status};
   CM_CUDA(cm::launch_mlp_up(up, tm_w1t, tm_x, s), "MLP up-projection launch");
   return CHIPMUNK_OK;
@@ -215,12 +216,12 @@ chipmunk_status mlp_down_impl(const chipmunk_mlp_args *a, void *ws, int *status,
   const int64_t k_pad = ceil_div(a->k, 128) * 128;
   const int bn = down_bn(a->D);
   cm::MlpDownParams dp{int(a->T), int(a->D), a->Bt, int(nb), int(k_pad), a->k, int(a->D / bn), bn,
-                       cm::kDownAccumulate, a->idx, static_cast<const uint16_t *>(a->b2), a->y_cache,
-                       static_cast<uint16_t *>(a->out), status};
+                       cm::kDownAccumulate, static_cast<const uint16_t *>(a->w2), int(a->H), a->idx,
+                       static_cast<const uint16_t *>(a->b2), a->y_cache, static_cast<uint16_t *>(a->out), status};
   CUtensorMap tm_d, tm_w2;
   if (a->k > 0) {
     CM_CHECK(map_blocks(&tm_d, ws, nb, k_pad, a->Bt, "delta workspace"));
-    CM_CHECK(map2d(&tm_w2, a->w2, a->H, a->D, 64, 1, "w2 gather"));
+    CM_CHECK(map2d(&tm_w2, a->w2, a->H, a->D, 64, 64, "w2"));
   }
   CM_CUDA(cm::launch_mlp_down(dp, tm_d, tm_w2, false, s), "MLP down-projection launch");
   return CHIPMUNK_OK;
@@ -309,10 +310,11 @@ chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, void *ws, size_
   const uint64_t cols = uint64_t(a->h) * 128;
   CUtensorMap tm_q, tm_k, tm_v;
   CM_CHECK(map2d(&tm_q, a->q, a->T, cols, 64, 128, "q"));
-  CM_CHECK(map2d(&tm_k, a->kk, a->T, cols, 64, 1, "k gather"));
-  CM_CHECK(map2d(&tm_v, a->v, a->T, cols, 64, 1, "v gather"));
-  cm::AttnParams p{int(a->T), a->h, int(nb), a->k, a->scale * 1.4426950408889634f, a->idx, a->m_c, a->l_c,
-                   a->acc_c, static_cast<uint16_t *>(a->o), nullptr, status};
+  CM_CHECK(map2d(&tm_k, a->kk, a->T, cols, 64, 128, "k"));
+  CM_CHECK(map2d(&tm_v, a->v, a->T, cols, 64, 128, "v"));
+  cm::AttnParams p{int(a->T), a->h, int(nb), a->k, a->scale * 1.4426950408889634f,
+                   static_cast<const uint16_t *>(a->kk), static_cast<const uint16_t *>(a->v), a->idx, a->m_c,
+                   a->l_c, a->acc_c, static_cast<uint16_t *>(a->o), nullptr, status};
   CM_CUDA(cm::launch_attn(cm::kAttnDelta, p, tm_q, tm_k, tm_v, s), "attention delta launch");
   return CHIPMUNK_OK;
 }
@@ -332,18 +334,18 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
     const int64_t nchunks = ceil_div(a->H, 128);
     const int bn = down_bn(a->D);
     CUtensorMap tm_w1t, tm_x, tm_a, tm_w2;
-    CM_CHECK(map2d(&tm_w1t, a->w1t, a->H, a->D, 64, 1, "w1t gather"));
+    CM_CHECK(map2d(&tm_w1t, a->w1t, a->H, a->D, 64, 128, "w1t"));
     CM_CHECK(map2d(&tm_x, a->x, a->T, a->D, 64, a->Bt, "x"));
     CM_CHECK(map_blocks(&tm_a, a->a_cache, nb, a->H, a->Bt, "activation cache"));
     CM_CHECK(map2d(&tm_w2, a->w2, a->H, a->D, 64, 64, "w2 tile"));
     cm::MlpUpParams up{int(a->T), int(a->D), int(a->H), int(a->H), a->Bt, int(nb), int(nchunks), int(nchunks * 128),
-                       r->first_step ? cm::kUpRefreshFirst : cm::kUpRefresh, nullptr,
-                       static_cast<const uint16_t *>(a->b1), static_cast<uint16_t *>(a->a_cache), nullptr, r->scores,
-                       status};
+                       r->first_step ? cm::kUpRefreshFirst : cm::kUpRefresh, static_cast<const uint16_t *>(a->w1t),
+                       nullptr, static_cast<const uint16_t *>(a->b1), static_cast<uint16_t *>(a->a_cache), nullptr,
+                       r->scores, status};
     CM_CUDA(cm::launch_mlp_up(up, tm_w1t, tm_x, s), "MLP refresh up-projection launch");
     cm::MlpDownParams dp{int(a->T), int(a->D), a->Bt, int(nb), int(a->H), int(a->H), int(a->D / bn), bn,
-                         cm::kDownOverwrite, nullptr, static_cast<const uint16_t *>(a->b2), a->y_cache,
-                         static_cast<uint16_t *>(a->out), status};
+                         cm::kDownOverwrite, static_cast<const uint16_t *>(a->w2), int(a->H), nullptr,
+                         static_cast<const uint16_t *>(a->b2), a->y_cache, static_cast<uint16_t *>(a->out), status};
     CM_CUDA(cm::launch_mlp_down(dp, tm_a, tm_w2, true, s), "MLP refresh down-projection launch");
     return topk_impl(r->scores, nb, a->H, a->H, a->k, a->idx, a->k, s);
   }
@@ -364,7 +366,8 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
     CM_CHECK(map2d(&tm_v, a->v, a->T, cols, 64, 128, "v tile"));
     float *lse = static_cast<float *>(ws);
     const float sl2 = a->scale * 1.4426950408889634f;
-    cm::AttnParams dense{int(a->T), a->h, int(nb), a->k, sl2, a->idx, a->m_c, a->l_c, a->acc_c,
+    cm::AttnParams dense{int(a->T), a->h, int(nb), a->k, sl2, static_cast<const uint16_t *>(a->kk),
+                         static_cast<const uint16_t *>(a->v), a->idx, a->m_c, a->l_c, a->acc_c,
                          static_cast<uint16_t *>(a->o), lse, status};
     CM_CUDA(cm::launch_attn(cm::kAttnDense, dense, tm_q, tm_k, tm_v, s), "attention refresh dense launch");
     cm::MassParams mp{int(a->T), a->h, int(nb), sl2, lse, r->scores, status};

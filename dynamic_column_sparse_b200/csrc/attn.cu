@@ -2,11 +2,13 @@
 // plus the dense passes of the refresh (full attention with row log-sum-exp,
 // attention mass per query block, complement partial).
 //
-// One CTA per (head, 128-query block). Warp 0 loads Q once and streams K/V in
-// chunks of 128 keys (TMA gather4 of the selected key rows on a sparse step,
-// tiled loads on the dense passes) through a two-stage ring. Warp 1 issues the
-// tcgen05 MMAs: S = Q K^T into one of two TMEM buffers, then O_tmp = P V into a
-// third. Warps 2..5 run the online softmax, one query row per thread: they
+// One CTA per (head, 128-query block). Q arrives once by a tiled TMA load; K
+// and V stream in chunks of 128 keys through a two-stage ring: on a sparse
+// step the producer warps 5-7 gather the selected key rows with 16-byte
+// cp.async (one warp instruction = two whole 256-byte key rows), on the dense
+// passes one thread issues tiled TMA loads. Warp 4 issues the tcgen05 MMAs:
+// S = Q K^T into one of two TMEM buffers, then O_tmp = P V into a third.
+// Warps 0-3 run the online softmax, one query row per thread: they
 // read S from TMEM, write P (bf16) into a 128-byte-swizzled shared tile that is
 // the A operand of the next P V, and fold each O_tmp into a register
 // accumulator rescaled by the running max. S of chunk i+1 is computed while the
@@ -19,7 +21,10 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp0 = 5;
+constexpr int kProducers = 96;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -74,8 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
+      mbar_init(&k_full[s], MODE == kAttnDelta ? kProducers : 1);
+      mbar_init(&v_full[s], MODE == kAttnDelta ? kProducers : 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 128);
@@ -86,12 +91,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kProdWarp0 && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -112,8 +117,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0 && nchunks > 0) {
+  if (warp >= kProdWarp0) {
+    const int pw = warp - kProdWarp0;
+    if (pw == 0 && lane == 0 && nchunks > 0) {
       mbar_arrive_expect_tx(q_full, kTileBytes);
       tma_load_2d(sQ, &tm_q, q_full, hh * 128, b * 128);
       tma_load_2d(sQ + 16384, &tm_q, q_full, hh * 128 + 64, b * 128);
@@ -124,22 +130,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t *dk = sK + s * kTileBytes;
       uint8_t *dv = sV + s * kTileBytes;
       if (MODE == kAttnDelta) {
-        int key[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) key[e] = __ldg(irow + min(i * 128 + lane * 4 + e, p.k - 1));
-        if (lane == 0) mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        __syncwarp();
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-          tma_gather4(dk + half * 16384 + lane * 512, &tm_k, &k_full[s], hh * 128 + half * 64, key[0], key[1], key[2],
-                      key[3]);
-        if (lane == 0) mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        __syncwarp();
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-          tma_gather4(dv + half * 16384 + lane * 512, &tm_v, &v_full[s], hh * 128 + half * 64, key[0], key[1], key[2],
-                      key[3]);
-      } else if (lane == 0) {
+        // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
+        const int c16 = lane & 15;
+        const uint32_t off_half = (c16 >> 3) * 16384;
+        const uint32_t k0 = smem_u32(dk), v0 = smem_u32(dv);
+        for (int qp = pw; qp < 64; qp += 3) {
+          const int r = 2 * qp + (lane >> 4);
+          int key = __ldg(irow + min(i * 128 + r, p.k - 1));
+          if (static_cast<unsigned>(key) >= static_cast<unsigned>(T)) {
+            atomicCAS(p.status, kDevOk, kDevBadIndex);
+            key = 0;
+          }
+          const size_t g = (static_cast<size_t>(key) * p.h + hh) * 128 + c16 * 8;
+          const uint32_t o = off_half + sw128_offset(r, c16 & 7);
+          cp_async_16(k0 + o, p.k_ptr + g);
+          cp_async_16(v0 + o, p.v_ptr + g);
+        }
+        cp_async_arrive_noinc(&k_full[s]);
+        cp_async_arrive_noinc(&v_full[s]);
+      } else if (pw == 0 && lane == 0) {
         mbar_arrive_expect_tx(&k_full[s], kTileBytes);
         tma_load_2d(dk, &tm_k, &k_full[s], hh * 128, i * 128);
         tma_load_2d(dk + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
@@ -149,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     if (nchunks > 0 && wait_warp(q_full, 0, p.status, abort_flag)) {
       tc_fence_after();
       const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
@@ -158,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = i & 1;
           if (!wait_warp(&k_full[s], (i >> 1) & 1, p.status, abort_flag)) break;
           if (!wait_warp(&s_free[s], ((i >> 1) & 1) ^ 1, p.status, abort_flag)) break;
+          if (MODE == kAttnDelta) fence_async_smem();
           tc_fence_after();
           if (lane == 0) {
             const uint32_t k0 = smem_u32(sK + s * kTileBytes);
@@ -176,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_warp(p_full, j & 1, p.status, abort_flag)) break;
           if (!wait_warp(&v_full[s], (j >> 1) & 1, p.status, abort_flag)) break;
           if (!wait_warp(o_free, (j & 1) ^ 1, p.status, abort_flag)) break;
+          fence_async_smem();
           tc_fence_after();
           if (lane == 0) {
             const uint32_t v0 = smem_u32(sV + s * kTileBytes);
@@ -209,20 +220,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      // bit e of live[c]: key slot i*128 + c*32 + e takes part in this pass
+      uint32_t live[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int base = i * 128 + c * 32;
+        const int lim = (MODE == kAttnDelta ? p.k : T) - base;
+        uint32_t m = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+        if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
+        live[c] = m;
+      }
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_off + sb * 128 + c * 32, v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int slot = i * 128 + c * 32 + e;
-          bool valid;
-          if (MODE == kAttnDelta) valid = slot < p.k;
-          else if (MODE == kAttnDense) valid = slot < T;
-          else valid = slot < T && !((mask[slot >> 5] >> (slot & 31)) & 1u);
-          if (valid) mx = fmaxf(mx, v[e] * sl2);
-        }
+        for (int e = 0; e < 32; ++e)
+          if ((live[c] >> e) & 1u) mx = fmaxf(mx, v[e] * sl2);
       }
       const float m_new = fmaxf(m2, mx);
       const float alpha = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - m_new);
@@ -256,11 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pe[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int slot = i * 128 + c * 32 + e + u;
-            bool valid;
-            if (MODE == kAttnDelta) valid = slot < p.k;
-            else if (MODE == kAttnDense) valid = slot < T;
-            else valid = slot < T && !((mask[slot >> 5] >> (slot & 31)) & 1u);
+            const bool valid = (live[c] >> (e + u)) & 1u;
             pe[u] = (valid && m2 != -INFINITY) ? exp2_approx(v[e + u] * sl2 - m2) : 0.f;
             l += pe[u];
           }
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // Attention mass of each key for one query block: D = K Q^T in TMEM (lane =
@@ -348,8 +359,9 @@ constexpr uint32_t kMKOff = 32768;        // 2 stages x 32 KB
 constexpr uint32_t kMBarOff = 98304;
 constexpr uint32_t kMLseOff = kMBarOff + 256;
 constexpr uint32_t kMSmem = 1024 + kMLseOff + 512 + 64;
+constexpr int kMassThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 column sums
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMassThreads, 1)
     attn_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const MassParams p) {
   constexpr uint32_t kIdesc = idesc_bf16(128, 128, false, false);
@@ -502,7 +514,7 @@ cudaError_t launch_attn_mass(const MassParams &p, const CUtensorMap &tm_q, const
                                        static_cast<int>(kMSmem));
   if (e != cudaSuccess) return e;
   const int64_t grid = static_cast<int64_t>(p.h) * p.nb;
-  attn_mass_kernel<<<static_cast<unsigned>(grid), kThreads, kMSmem, s>>>(tm_q, tm_k, p);
+  attn_mass_kernel<<<static_cast<unsigned>(grid), kMassThreads, kMSmem, s>>>(tm_q, tm_k, p);
   return cudaGetLastError();
 }
 

@@ -34,6 +34,7 @@ enum MlpUpMode : int { kUpDelta = 0, kUpRefresh = 1, kUpRefreshFirst = 2 };
 // epilogue. One CTA per (token block, chunk of 128 selected columns).
 struct MlpUpParams {
   int T, D, H, k, Bt, nb, nchunks, k_pad, mode;
+  const uint16_t *w1t;    // [H][D] (rows gathered on a sparse step)
   const int32_t *idx;     // [nb][k] (sparse step)
   const uint16_t *b1;     // [H]
   uint16_t *a_cache;      // [nb][H][Bt]
@@ -41,8 +42,8 @@ struct MlpUpParams {
   float *scores;          // [nb][H] (refresh)
   int *status;
 };
-cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t_gather, const CUtensorMap &tm_x,
-                          cudaStream_t s);
+// tm_w1t: tile map over W1^T [H][D] (box 64 x 128), read on a refresh only.
+cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s);
 
 enum MlpDownMode : int { kDownAccumulate = 0, kDownOverwrite = 1 };
 
@@ -51,13 +52,15 @@ enum MlpDownMode : int { kDownAccumulate = 0, kDownOverwrite = 1 };
 // cache (refresh, all rows). One CTA per (token block, slice of BN columns).
 struct MlpDownParams {
   int T, D, Bt, nb, krows, k, n_slices, bn, mode;
+  const uint16_t *w2;     // [H][D] (rows gathered on a sparse step)
+  int H;
   const int32_t *idx;     // [nb][k] (sparse step)
   const uint16_t *b2;     // [D] (refresh)
   float *y_cache;         // [T][D]
   uint16_t *out;          // [T][D] or nullptr
   int *status;
 };
-// tm_a: 3-D map over A [nb][rows][Bt]; tm_w2: gather4 map (sparse) or tile map (dense) over W2 [H][D].
+// tm_a: 3-D map over A [nb][rows][Bt]; tm_w2: tile map over W2 [H][D] (box 64 x 64), read on a refresh only.
 cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
                             cudaStream_t s);
 
@@ -68,6 +71,7 @@ enum AttnMode : int { kAttnDelta = 0, kAttnDense = 1, kAttnComplement = 2 };
 struct AttnParams {
   int T, h, nb, k;
   float scale_log2;       // logit scale * log2(e)
+  const uint16_t *k_ptr, *v_ptr;  // [T][h][128] (key rows gathered on a sparse step)
   const int32_t *idx;     // [h][nb][k]
   float *m_c, *l_c, *acc_c;  // [h][T], [h][T], [h][T][128]
   uint16_t *o;            // [T][h][128]

@@ -1,23 +1,27 @@
 // mlp.cu - gathered-column MLP kernels of the sparse delta step and the refresh.
 //
 // Kernel 1 (mlp_up): one CTA per (token block b, chunk of 128 selected hidden
-// columns). The selected rows of W1^T are gathered from global memory into
-// 128-byte-swizzled shared-memory tiles with TMA gather4 (four arbitrary rows
-// per instruction), the token block of x arrives by a tiled TMA load, and one
-// thread issues tcgen05 bf16 MMAs accumulating D[col][token] in TMEM. The
-// epilogue warps own one hidden column each (one TMEM lane) and all Bt tokens
-// of it, so the activation cache run a_cache[b][c][0..Bt) and the delta row
-// are read and written as whole contiguous runs.
+// columns). The 128 selected rows of W1^T are gathered into a 128-byte-
+// swizzled shared tile by four producer warps with 16-byte cp.async (each
+// warp instruction moves four whole 128-byte row segments); on a refresh,
+// where the rows are consecutive, one TMA tile load brings them instead. The
+// token block of x arrives by a tiled TMA load. One thread issues tcgen05 bf16
+// MMAs accumulating D[col][token] in TMEM. The epilogue warps own one hidden
+// column each (one TMEM lane) and all Bt tokens of it, so the activation cache
+// run a_cache[b][c][0..Bt) and the delta row are read and written as whole
+// contiguous runs.
 //
 // Kernel 2 (mlp_down): one CTA per (token block b, slice of BN model columns).
-// The K dimension runs over the selected hidden units: the delta rows come
-// from the workspace by tiled TMA, the matching W2 rows are gathered with TMA
-// gather4; both operands are MN-major. The epilogue adds the fp32 result into
-// the output cache (or overwrites it with result + b2 on a refresh) and writes
-// the bf16 layer output.
+// K runs over the selected hidden units: the delta rows come from the
+// workspace by tiled TMA, the matching W2 rows are gathered by the producer
+// warps with cp.async (one warp instruction = whole row segments); both
+// operands are MN-major. The epilogue adds the fp32 result into the output
+// cache (or overwrites it with result + b2 on a refresh) and writes the bf16
+// layer output.
 //
-// Warp roles in both kernels: warp 0 = TMA producer, warp 1 = MMA issuer
-// (and TMEM owner), warps 2..5 = epilogue (TMEM lane quadrant = warp % 4).
+// Warp roles: warps 0-3 = producers (thread 0 also issues the TMA tile
+// loads), warp 4 = MMA issuer and TMEM owner, warps 5-8 = epilogue (TMEM lane
+// quadrant = warp % 4).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -26,7 +30,9 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 288;
+constexpr int kProducers = 128;
+constexpr int kMmaWarp = 4;
 constexpr int kBK = 64;  // K elements per pipeline stage = one 128-byte swizzle row
 
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
@@ -44,7 +50,7 @@ struct UpCfg {
   static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
 };
 
-template <int BT>
+template <int BT, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 1)
     mlp_up_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
                   const MlpUpParams p) {
@@ -69,18 +75,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], DENSE ? 1 : 1 + kProducers);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (threadIdx.x == 32) {
     prefetch_tmap(&tm_w1t);
     prefetch_tmap(&tm_x);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, BT);
     tmem_relinquish();
   }
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int c;
     if (sparse) {
       c = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
-      if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the cache
+      if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights / cache
         atomicCAS(p.status, kDevOk, kDevBadIndex);
         c = 0;
       }
@@ -104,18 +110,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int nk = p.D / kBK;
 
-  if (warp == 0) {
+  if (warp < 4) {
+    // producers: thread pt moves 16-byte chunk (pt & 7) of rows i*16 + (pt >> 3), i = 0..7
+    const int pt = threadIdx.x;
+    const uint16_t *src_row[8];
+    uint32_t dst_off[8];
+    if (!DENSE) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = i * 16 + (pt >> 3);
+        src_row[i] = p.w1t + static_cast<size_t>(rows[r]) * p.D + (pt & 7) * 8;
+        dst_off[i] = sw128_offset(r, pt & 7);
+      }
+    }
+    const uint32_t a_base = smem_u32(sA);
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % C::kStages;
       const uint32_t ph = (kb / C::kStages) & 1;
       if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], C::kABytes + C::kBBytes);
-      __syncwarp();
-      tma_gather4(sA + s * C::kABytes + lane * 512, &tm_w1t, &full[s], kb * kBK, rows[4 * lane], rows[4 * lane + 1],
-                  rows[4 * lane + 2], rows[4 * lane + 3]);
-      if (lane == 0) tma_load_2d(sB + s * C::kBBytes, &tm_x, &full[s], kb * kBK, b * BT);
+      if (pt == 0) {
+        mbar_arrive_expect_tx(&full[s], C::kBBytes + (DENSE ? C::kABytes : 0));
+        tma_load_2d(sB + s * C::kBBytes, &tm_x, &full[s], kb * kBK, b * BT);
+        if (DENSE) tma_load_2d(sA + s * C::kABytes, &tm_w1t, &full[s], kb * kBK, chunk * 128);
+      }
+      if (!DENSE) {
+        const uint32_t stage = a_base + s * C::kABytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
+        cp_async_arrive_noinc(&full[s]);
+      }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % C::kStages;
@@ -124,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      if (!DENSE) fence_async_smem();
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = smem_u32(sA + s * C::kABytes);
@@ -160,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + tq * 32, acc);
         uint4 oldv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
                          make_uint4(0, 0, 0, 0)};
-        if (valid_j) {
+        if (valid_j && !(first && !sparse)) {
           const uint4 *src = reinterpret_cast<const uint4 *>(arow + tq * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) oldv[v] = src[v];
@@ -205,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, BT);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, BT);
 }
 
 template <int BN>
@@ -223,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const MlpDownParams p) {
   using C = DownCfg<BN>;
   constexpr uint32_t kIdesc = idesc_bf16(128, BN, true, true);
-  constexpr uint32_t kTx = (BT / 64) * 8192 + C::kBBytes;
+  constexpr uint32_t kATx = (BT / 64) * 8192;
+  constexpr int kChunksPerRow = BN / 8;               // 16-byte chunks of one gathered W2 row segment
+  constexpr int kRowsPerInstr = 32 / kChunksPerRow;   // rows one warp instruction covers
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
@@ -244,18 +272,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], DENSE ? 1 : 1 + kProducers);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (threadIdx.x == 32) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_w2);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
@@ -272,14 +300,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < 4) {
+    // producers: warp pw gathers W2 rows pw*16 .. pw*16+15 of each 64-row stage
+    const int pt = threadIdx.x, pw = warp;
     const int32_t *irow = DENSE ? nullptr : p.idx + static_cast<size_t>(b) * p.k;
+    const int csub = lane % kChunksPerRow;           // chunk of the row segment this lane moves
+    const int rsub = lane / kChunksPerRow;           // row within one instruction
+    const uint32_t b_base = smem_u32(sB);
+    auto load_idx = [&](int kb) -> int {             // lane < 16: index of row pw*16 + lane of stage kb
+      int c = 0;
+      if (!DENSE && lane < 16 && kb < nk) {
+        c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
+        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
+          atomicCAS(p.status, kDevOk, kDevBadIndex);
+          c = 0;
+        }
+      }
+      return c;
+    };
+    int c_cur = load_idx(0);
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % C::kStages;
       const uint32_t ph = (kb / C::kStages) & 1;
+      const int c_next = load_idx(kb + 1);
       if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], kTx);
+      if (pt == 0) {
+        mbar_arrive_expect_tx(&full[s], kATx + (DENSE ? C::kBBytes : 0));
 #pragma unroll
         for (int mt = 0; mt < BT / 64; ++mt)
           tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &full[s], mt * 64, kb * kBK, b);
@@ -289,21 +335,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &full[s], n0 + ns * 64, kb * kBK);
         }
       }
-      __syncwarp();
       if (!DENSE) {
-        // 16 groups of 4 rows per 64-column slab; lane l issues groups l, l+32, ...
-        for (int g = lane; g < 16 * (BN / 64); g += 32) {
-          const int ns = g >> 4, grp = g & 15;
-          const int j0 = kb * kBK + grp * 4;
-          int c[4];
+        const uint32_t stage = b_base + s * C::kBBytes;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) c[e] = __ldg(irow + min(j0 + e, p.k - 1));
-          tma_gather4(sB + s * C::kBBytes + ns * 8192 + grp * 512, &tm_w2, &full[s], n0 + ns * 64, c[0], c[1], c[2],
-                      c[3]);
+        for (int i = 0; i < 16 / kRowsPerInstr; ++i) {
+          const int rr = i * kRowsPerInstr + rsub;   // 0..15 within this warp's rows
+          const int r = pw * 16 + rr;                // row of the stage
+          const int c = __shfl_sync(0xffffffffu, c_cur, rr);
+          const int slab = csub >> 3, cc = csub & 7;
+          cp_async_16(stage + slab * 8192 + sw128_offset(r, cc), p.w2 + static_cast<size_t>(c) * p.D + n0 + csub * 8);
         }
+        cp_async_arrive_noinc(&full[s]);
       }
+      c_cur = c_next;
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % C::kStages;
@@ -312,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      if (!DENSE) fence_async_smem();
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = smem_u32(sA + s * C::kABytes);
@@ -372,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, BN);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, BN);
 }
 
 // out = bf16(y) when a sparse step selects nothing
@@ -389,13 +436,13 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
-template <int BT>
+template <int BT, bool DENSE>
 cudaError_t launch_up_t(const MlpUpParams &p, const CUtensorMap &w, const CUtensorMap &x, cudaStream_t s) {
   using C = UpCfg<BT>;
-  cudaError_t e = set_smem(mlp_up_kernel<BT>, C::kSmem);
+  cudaError_t e = set_smem(mlp_up_kernel<BT, DENSE>, C::kSmem);
   if (e != cudaSuccess) return e;
   const int64_t grid = static_cast<int64_t>(p.nb) * p.nchunks;
-  mlp_up_kernel<BT><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(w, x, p);
+  mlp_up_kernel<BT, DENSE><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(w, x, p);
   return cudaGetLastError();
 }
 
@@ -421,11 +468,11 @@ cudaError_t launch_down_bn(const MlpDownParams &p, const CUtensorMap &a, const C
 
 }  // namespace
 
-cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t_gather, const CUtensorMap &tm_x,
-                          cudaStream_t s) {
+cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s) {
   if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
-  if (p.Bt == 128) return launch_up_t<128>(p, tm_w1t_gather, tm_x, s);
-  if (p.Bt == 64) return launch_up_t<64>(p, tm_w1t_gather, tm_x, s);
+  const bool dense = p.mode != kUpDelta;
+  if (p.Bt == 128) return dense ? launch_up_t<128, true>(p, tm_w1t, tm_x, s) : launch_up_t<128, false>(p, tm_w1t, tm_x, s);
+  if (p.Bt == 64) return dense ? launch_up_t<64, true>(p, tm_w1t, tm_x, s) : launch_up_t<64, false>(p, tm_w1t, tm_x, s);
   return cudaErrorInvalidValue;
 }
 

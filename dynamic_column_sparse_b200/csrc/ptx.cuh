@@ -121,6 +121,25 @@ __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *tm, ui
       : "memory");
 }
 
+// 16 bytes global -> shared, cached in L2 only. Completion is tracked by
+// cp_async_arrive_noinc on an mbarrier.
+__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+
+// The mbarrier receives one arrival once every cp.async this thread issued
+// so far has landed (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a tile of
+// 128-byte rows with the 128-byte swizzle (chunk index XOR row mod 8), as TMA
+// writes it and the UMMA descriptors read it.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 // ----------------------------------------------------------------- tcgen05
 
 // Whole warp. Writes the TMEM base address to *dst (shared memory).
