@@ -21,73 +21,100 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 5;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxThreads = 256;   // warps 0-7: two warps per TMEM lane quadrant, one per half of the columns
+constexpr int kMmaWarp = 8;
+constexpr int kProdWarp0 = 9;          // warps 9-11
 constexpr int kProducers = 96;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two 64-column swizzle halves)
+constexpr float kRescaleLog2 = 8.0f;     // O and l are rescaled only when the row max grows by more than 2^8
 
-constexpr uint32_t kQOff = 0;             // Q: two 64-column halves of [128 rows][128 B]
-constexpr uint32_t kKOff = 32768;         // K: 2 stages x 32 KB
-constexpr uint32_t kVOff = 98304;         // V: 2 stages x 32 KB
-constexpr uint32_t kPOff = 163840;        // P: two 64-key halves of [128 rows][128 B]
-constexpr uint32_t kBarOff = 196608;
-constexpr uint32_t kMaskOff = kBarOff + 256;
-constexpr uint32_t kTileBytes = 32768;
+// Shared memory: Q | K[2] | V[2] | P | barriers | key-index ring [2][128] |
+// row-max exchange [2][2][128] | row-sum exchange [2][2][128] | key mask (complement pass).
+struct AttnCfg {
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKOff = kTileBytes;
+  static constexpr uint32_t kVOff = kKOff + 2 * kTileBytes;
+  static constexpr uint32_t kPOff = kVOff + 2 * kTileBytes;
+  static constexpr uint32_t kBarOff = kPOff + kTileBytes;
+  static constexpr uint32_t kIdxOff = kBarOff + 256;
+  static constexpr uint32_t kXmaxOff = kIdxOff + 2 * 128 * 4;
+  static constexpr uint32_t kXsumOff = kXmaxOff + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kMaskOff = kXsumOff + 2 * 2 * 128 * 4;
+};
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
   const bool ok = mbar_wait(bar, parity, status, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
 
+// exp2 of 64 values in place: one in every `kFmaEvery` on the FMA pipe, the rest on MUFU
+constexpr int kFmaEvery = 5;
+
+// Persistent: each CTA walks tiles (head, 128-query block) blockIdx.x,
+// blockIdx.x + gridDim.x, ...; every tile has the same number of key chunks,
+// so all roles index chunks by one running counter g.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnCfg;
   constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16(128, 128, false, true);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
-  uint8_t *sQ = smem + kQOff;
-  uint8_t *sK = smem + kKOff;
-  uint8_t *sV = smem + kVOff;
-  uint8_t *sP = smem + kPOff;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff);
+  uint8_t *sQ = smem + C::kQOff;
+  uint8_t *sK = smem + C::kKOff;
+  uint8_t *sV = smem + C::kVOff;
+  uint8_t *sP = smem + C::kPOff;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
   uint64_t *q_full = bars + 0;
-  uint64_t *k_full = bars + 1;    // [2]
-  uint64_t *v_full = bars + 3;    // [2]
-  uint64_t *kv_empty = bars + 5;  // [2]
-  uint64_t *s_full = bars + 7;    // [2]
-  uint64_t *s_free = bars + 9;    // [2]
-  uint64_t *p_full = bars + 11;
-  uint64_t *o_full = bars + 12;
-  uint64_t *o_free = bars + 13;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+  uint64_t *q_empty = bars + 1;
+  uint64_t *k_full = bars + 2;     // [2]
+  uint64_t *v_full = bars + 4;     // [2]
+  uint64_t *kv_empty = bars + 6;   // [2]
+  uint64_t *s_full = bars + 8;     // [2]
+  uint64_t *s_empty = bars + 10;   // [2]
+  uint64_t *o_full = bars + 12;    // [2]
+  uint64_t *o_empty = bars + 14;   // [2]
+  uint64_t *p_full = bars + 16;
+  uint64_t *p_empty = bars + 17;
+  uint64_t *pair_bar = bars + 18;  // [4]: the two softmax warps of a lane quadrant exchange row partials
+  uint64_t *kidx_bar = bars + 22;  // producers: a chunk's keys are staged
+  uint64_t *mask_bar = bars + 23;  // softmax warps: complement mask steps
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  uint32_t *mask = reinterpret_cast<uint32_t *>(smem + kMaskOff);
+  int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [2][128] selected keys of a chunk
+  float *xmax = reinterpret_cast<float *>(smem + C::kXmaxOff);   // [2][2][128] partial row maxima
+  float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
+  uint32_t *mask = reinterpret_cast<uint32_t *>(smem + C::kMaskOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  const int hh = blockIdx.x % p.h;
-  const int b = blockIdx.x / p.h;
   const int T = p.T;
+  const int ntiles = p.h * p.nb;
   const int nkeys = MODE == kAttnDelta ? p.k : T;
   const int nchunks = (nkeys + 127) / 128;
-  const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], MODE == kAttnDelta ? kProducers : 1);
       mbar_init(&v_full[s], MODE == kAttnDelta ? kProducers : 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
+      mbar_init(&s_empty[s], kSoftmaxThreads);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], kSoftmaxThreads);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
-    mbar_init(o_free, 128);
+    mbar_init(p_full, kSoftmaxThreads);
+    mbar_init(p_empty, 1);
+    for (int qd = 0; qd < 4; ++qd) mbar_init(&pair_bar[qd], 64);
+    mbar_init(kidx_bar, kProducers);
+    mbar_init(mask_bar, kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -100,73 +127,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (MODE == kAttnComplement) {
-    const int nwords = (T + 31) >> 5;
-    for (int w = threadIdx.x; w < nwords; w += kThreads) mask[w] = 0u;
-    __syncthreads();
-    for (int j = threadIdx.x; j < p.k; j += kThreads) {
-      const int key = __ldg(irow + j);
-      if (static_cast<unsigned>(key) < static_cast<unsigned>(T))
-        atomicOr(&mask[key >> 5], 1u << (key & 31));
-      else
-        atomicCAS(p.status, kDevOk, kDevBadIndex);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = *tmem_slot;   // S[0] at column 0, S[1] at 128, O[0] at 256, O[1] at 384
 
   if (warp >= kProdWarp0) {
+    // ------------------------------------------------------------ producers
     const int pw = warp - kProdWarp0;
-    if (pw == 0 && lane == 0 && nchunks > 0) {
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_2d(sQ, &tm_q, q_full, hh * 128, b * 128);
-      tma_load_2d(sQ + 16384, &tm_q, q_full, hh * 128 + 64, b * 128);
-    }
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i & 1;
-      if (!wait_warp(&kv_empty[s], ((i >> 1) & 1) ^ 1, p.status, abort_flag)) break;
-      uint8_t *dk = sK + s * kTileBytes;
-      uint8_t *dv = sV + s * kTileBytes;
-      if (MODE == kAttnDelta) {
-        // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
-        const int c16 = lane & 15;
-        const uint32_t off_half = (c16 >> 3) * 16384;
-        const uint32_t k0 = smem_u32(dk), v0 = smem_u32(dv);
-        for (int qp = pw; qp < 64; qp += 3) {
-          const int r = 2 * qp + (lane >> 4);
-          int key = __ldg(irow + min(i * 128 + r, p.k - 1));
-          if (static_cast<unsigned>(key) >= static_cast<unsigned>(T)) {
-            atomicCAS(p.status, kDevOk, kDevBadIndex);
-            key = 0;
-          }
-          const size_t g = (static_cast<size_t>(key) * p.h + hh) * 128 + c16 * 8;
-          const uint32_t o = off_half + sw128_offset(r, c16 & 7);
-          cp_async_16(k0 + o, p.k_ptr + g);
-          cp_async_16(v0 + o, p.v_ptr + g);
-        }
-        cp_async_arrive_noinc(&k_full[s]);
-        cp_async_arrive_noinc(&v_full[s]);
-      } else if (pw == 0 && lane == 0) {
-        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_2d(dk, &tm_k, &k_full[s], hh * 128, i * 128);
-        tma_load_2d(dk + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
-        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-        tma_load_2d(dv, &tm_v, &v_full[s], hh * 128, i * 128);
-        tma_load_2d(dv + 16384, &tm_v, &v_full[s], hh * 128 + 64, i * 128);
+    const int pt = threadIdx.x - kProdWarp0 * 32;  // 0..95
+    // selected keys of chunk i of tile `tile`, rows pt and pt + 96 (the latter for pt < 32)
+    auto load_keys = [&](int tile, int i, int &ka, int &kb2) {
+      const int hh = tile % p.h, b = tile / p.h;
+      const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
+      ka = __ldg(irow + min(i * 128 + pt, p.k - 1));
+      kb2 = pt < 32 ? __ldg(irow + min(i * 128 + pt + 96, p.k - 1)) : 0;
+      if (static_cast<unsigned>(ka) >= static_cast<unsigned>(T) || static_cast<unsigned>(kb2) >= static_cast<unsigned>(T)) {
+        atomicCAS(p.status, kDevOk, kDevBadIndex);
+        ka = static_cast<unsigned>(ka) >= static_cast<unsigned>(T) ? 0 : ka;
+        kb2 = static_cast<unsigned>(kb2) >= static_cast<unsigned>(T) ? 0 : kb2;
       }
-      __syncwarp();
+    };
+    int ka = 0, kb2 = 0;
+    if (MODE == kAttnDelta && nchunks > 0 && static_cast<int>(blockIdx.x) < ntiles) load_keys(blockIdx.x, 0, ka, kb2);
+    uint32_t kidx_phase = 0;
+    int tl = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
+      if (nchunks == 0) continue;
+      const int hh = tile % p.h, b = tile / p.h;
+      if (pw == 0) {
+        if (!wait_warp(q_empty, (tl & 1) ^ 1, p.status, abort_flag)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, kTileBytes);
+          tma_load_2d(sQ, &tm_q, q_full, hh * 128, b * 128);
+          tma_load_2d(sQ + 16384, &tm_q, q_full, hh * 128 + 64, b * 128);
+        }
+        __syncwarp();
+      }
+      for (int i = 0; i < nchunks; ++i) {
+        const int g = tl * nchunks + i, s = g & 1;
+        if (!wait_warp(&kv_empty[s], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t *dk = sK + s * kTileBytes;
+        uint8_t *dv = sV + s * kTileBytes;
+        if (MODE == kAttnDelta) {
+          // stage this chunk's keys, then fetch the next chunk's while the copies go out
+          int *ks = kidx + s * 128;
+          ks[pt] = ka;
+          if (pt < 32) ks[pt + 96] = kb2;
+          mbar_arrive(kidx_bar);
+          if (!wait_warp(kidx_bar, kidx_phase & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++kidx_phase;
+          {
+            int nt = tile, ni = i + 1;
+            if (ni == nchunks) {
+              ni = 0;
+              nt = tile + gridDim.x;
+            }
+            if (nt < ntiles) load_keys(nt, ni, ka, kb2);
+          }
+          // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
+          const int c16 = lane & 15;
+          const uint32_t off_half = (c16 >> 3) * 16384;
+          const uint32_t k0 = smem_u32(dk), v0 = smem_u32(dv);
+          for (int qp = pw; qp < 64; qp += 3) {
+            const int r = 2 * qp + (lane >> 4);
+            const int key = ks[r];
+            const size_t gsrc = (static_cast<size_t>(key) * p.h + hh) * 128 + c16 * 8;
+            const uint32_t o = off_half + sw128_offset(r, c16 & 7);
+            cp_async_16(k0 + o, p.k_ptr + gsrc);
+            cp_async_16(v0 + o, p.v_ptr + gsrc);
+          }
+          cp_async_arrive_noinc(&k_full[s]);
+          cp_async_arrive_noinc(&v_full[s]);
+        } else if (pw == 0 && lane == 0) {
+          mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+          tma_load_2d(dk, &tm_k, &k_full[s], hh * 128, i * 128);
+          tma_load_2d(dk + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
+          mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+          tma_load_2d(dv, &tm_v, &v_full[s], hh * 128, i * 128);
+          tma_load_2d(dv + 16384, &tm_v, &v_full[s], hh * 128 + 64, i * 128);
+        }
+        __syncwarp();
+      }
     }
   } else if (warp == kMmaWarp) {
-    if (nchunks > 0 && wait_warp(q_full, 0, p.status, abort_flag)) {
-      tc_fence_after();
-      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
-      for (int i = 0; i <= nchunks; ++i) {
+    // ------------------------------------------------------------ MMA issuer
+    int tl = 0;
+    bool ok = true;
+    const uint32_t p0 = smem_u32(sP), q0 = smem_u32(sQ);
+    for (int tile = blockIdx.x; tile < ntiles && ok && nchunks > 0; tile += gridDim.x, ++tl) {
+      const int ob = tl & 1;
+      const uint32_t tO = tmem + 256 + ob * 128;
+      if (!wait_warp(q_full, tl & 1, p.status, abort_flag)) break;
+      if (!wait_warp(&o_empty[ob], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
+      for (int i = 0; i <= nchunks && ok; ++i) {
         if (i < nchunks) {
-          const int s = i & 1;
-          if (!wait_warp(&k_full[s], (i >> 1) & 1, p.status, abort_flag)) break;
-          if (!wait_warp(&s_free[s], ((i >> 1) & 1) ^ 1, p.status, abort_flag)) break;
+          const int g = tl * nchunks + i, s = g & 1;
+          if (!wait_warp(&k_full[s], (g >> 1) & 1, p.status, abort_flag) ||
+              !wait_warp(&s_empty[s], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
           if (MODE == kAttnDelta) fence_async_smem();
           tc_fence_after();
           if (lane == 0) {
@@ -178,170 +246,238 @@ __global__ void __launch_bounds__(kThreads, 1)
                         kk > 0);
             }
             umma_commit(&s_full[s]);
+            if (i == nchunks - 1) umma_commit(q_empty);
           }
           __syncwarp();
         }
         if (i >= 1) {
-          const int j = i - 1, s = j & 1;
-          if (!wait_warp(p_full, j & 1, p.status, abort_flag)) break;
-          if (!wait_warp(&v_full[s], (j >> 1) & 1, p.status, abort_flag)) break;
-          if (!wait_warp(o_free, (j & 1) ^ 1, p.status, abort_flag)) break;
+          const int j = i - 1, g = tl * nchunks + j, s = g & 1;
+          if (!wait_warp(p_full, g & 1, p.status, abort_flag) ||
+              !wait_warp(&v_full[s], (g >> 1) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
           fence_async_smem();
           tc_fence_after();
           if (lane == 0) {
             const uint32_t v0 = smem_u32(sV + s * kTileBytes);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              umma_bf16(tmem + 256, sdesc_sw128(p0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV, kk > 0);
-            }
-            umma_commit(o_full);
+            for (int kk = 0; kk < 8; ++kk)
+              umma_bf16(tO, sdesc_sw128(p0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV, (j | kk) != 0);
             umma_commit(&kv_empty[s]);
+            umma_commit(p_empty);
+            if (j == nchunks - 1) umma_commit(&o_full[ob]);
           }
           __syncwarp();
         }
       }
     }
   } else {
-    const int q = warp & 3;
+    // ------------------------------------------------------------ softmax + epilogue (warps 0-7)
+    // warp w: TMEM lane quadrant w & 3 (query rows), column half w >> 2 (keys 64h.. of S, dims 64h.. of O)
+    const int q = warp & 3, half = warp >> 2;
     const int r = q * 32 + lane;
-    const int gi = b * 128 + r;
+    const int st = threadIdx.x;  // 0..255
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float sl2 = p.scale_log2;
-    float o_acc[128];
-#pragma unroll
-    for (int e = 0; e < 128; ++e) o_acc[e] = 0.f;
-    float m2 = -INFINITY, l = 0.f;
+    uint32_t pair_phase = 0, mask_phase = 0;
+    // both warps of the quadrant have written their partial; bounded wait
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&pair_bar[q]);
+      const bool r2 = wait_warp(&pair_bar[q], pair_phase & 1, p.status, abort_flag);
+      ++pair_phase;
+      return r2;
+    };
+    auto mask_sync = [&]() -> bool {
+      mbar_arrive(mask_bar);
+      const bool r2 = wait_warp(mask_bar, mask_phase & 1, p.status, abort_flag);
+      ++mask_phase;
+      return r2;
+    };
+    int tl = 0;
     bool ok = true;
-    for (int i = 0; i < nchunks && ok; ++i) {
-      const int sb = i & 1;
-      if (!wait_warp(&s_full[sb], (i >> 1) & 1, p.status, abort_flag)) {
-        ok = false;
-        break;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
+      const int hh = tile % p.h, b = tile / p.h;
+      const int gi = b * 128 + r;
+      const int ob = tl & 1;
+      const uint32_t tO = tmem + lane_off + 256 + ob * 128 + half * 64;
+      if (MODE == kAttnComplement) {
+        // mask of the keys this tile's block selected
+        const int nwords = (T + 31) >> 5;
+        if (!mask_sync()) break;   // every softmax warp is done with the previous tile's mask
+        for (int w = st; w < nwords; w += kSoftmaxThreads) mask[w] = 0u;
+        if (!mask_sync()) break;
+        const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
+        for (int j = st; j < p.k; j += kSoftmaxThreads) {
+          const int key = __ldg(irow + j);
+          if (static_cast<unsigned>(key) < static_cast<unsigned>(T))
+            atomicOr(&mask[key >> 5], 1u << (key & 31));
+          else
+            atomicCAS(p.status, kDevOk, kDevBadIndex);
+        }
+        if (!mask_sync()) break;
       }
-      tc_fence_after();
-      // bit e of live[c]: key slot i*128 + c*32 + e takes part in this pass
-      uint32_t live[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int base = i * 128 + c * 32;
-        const int lim = (MODE == kAttnDelta ? p.k : T) - base;
-        uint32_t m = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-        if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
-        live[c] = m;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + sb * 128 + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if ((live[c] >> e) & 1u) mx = fmaxf(mx, v[e] * sl2);
-      }
-      const float m_new = fmaxf(m2, mx);
-      const float alpha = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - m_new);
-      if (i >= 1) {
-        if (!wait_warp(o_full, (i - 1) & 1, p.status, abort_flag)) {
+      float m_used = -INFINITY, l = 0.f;   // m_used in log2 units of the scaled logits
+      for (int i = 0; i < nchunks; ++i) {
+        const int g = tl * nchunks + i, s = g & 1;
+        if (!wait_warp(&s_full[s], (g >> 1) & 1, p.status, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + 256 + c * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] += v[e];
-        }
+        float sv[64];
+        tmem_ld32_async(tmem + lane_off + s * 128 + half * 64, sv);
+        tmem_ld32_async(tmem + lane_off + s * 128 + half * 64 + 32, sv + 32);
+        tmem_wait_ld_regs(sv);
+        reg_fence32(sv + 32);
         tc_fence_before();
-        mbar_arrive(o_free);
-      }
+        mbar_arrive(&s_empty[s]);  // S now lives in registers: the buffer can take S of chunk g + 2
+        // keys of this half that take part: bits of live[0] (keys 64h..64h+31) and live[1]
+        uint32_t live[2];
 #pragma unroll
-      for (int e = 0; e < 128; ++e) o_acc[e] *= alpha;
-      l *= alpha;
-      m2 = m_new;
+        for (int c = 0; c < 2; ++c) {
+          const int base = i * 128 + half * 64 + c * 32;
+          const int lim = nkeys - base;
+          uint32_t m = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+          if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
+          live[c] = m;
+        }
+        if ((live[0] & live[1]) != 0xffffffffu) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + sb * 128 + c * 32, v);
-        uint32_t pk[16];
+          for (int e = 0; e < 64; ++e)
+            if (!((live[e >> 5] >> (e & 31)) & 1u)) sv[e] = -INFINITY;
+        }
+        float mxp[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pe[2];
+        for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const bool valid = (live[c] >> (e + u)) & 1u;
-            pe[u] = (valid && m2 != -INFINITY) ? exp2_approx(v[e + u] * sl2 - m2) : 0.f;
-            l += pe[u];
+        for (int e = 0; e < 64; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], sv[e]);
+        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        // combine with the other half of the row
+        float *xm = xmax + (s * 2) * 128;
+        xm[half * 128 + r] = mx;
+        if (!pair_sync()) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, xm[(half ^ 1) * 128 + r]) * sl2;
+        const float m_new = fmaxf(m_used, mx);
+        // lazy rescale: only when the max grows by more than 2^8 over the one in use
+        const bool need = m_used != -INFINITY && m_new > m_used + kRescaleLog2;
+        if (m_used == -INFINITY) m_used = m_new;
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds P V of the earlier chunks: wait for the last of them, then scale this half in TMEM
+          if (!wait_warp(p_empty, (g & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
           }
-          pk[e / 2] = pack_bf16x2(pe[0], pe[1]);
-        }
-        uint8_t *prow = sP + (c >> 1) * 16384 + r * 128;
+          tc_fence_after();
+          const float alpha = need ? exp2_approx(m_used - m_new) : 1.f;
+          if (need) {
+            l *= alpha;
+            m_used = m_new;
+          }
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            float ov[32];
+            tmem_ld32(tO + c * 32, ov);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int cc = (c & 1) * 4 + u;
-          *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(tO + c * 32, ov);
+          }
+          tmem_wait_st();
         }
+        // p = 2^(s * scale_log2 - m); masked keys hold -inf and give 0
+        const float mneg = (m_used == -INFINITY) ? 0.f : -m_used;
+        float lp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const float x = fmaf(sv[e], sl2, mneg);
+          sv[e] = (e % kFmaEvery == kFmaEvery - 1) ? exp2_fma(x) : exp2_approx(x);
+          lp[e & 3] += sv[e];
+        }
+        l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+        // P of the previous chunk must have been consumed before it is overwritten
+        if (!wait_warp(p_empty, (g & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t *prow = sP + half * 16384 + r * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {  // 16-byte chunk c8 = keys 64h + 8*c8 .. +7
+          const float *pv = sv + 8 * c8;
+          *reinterpret_cast<uint4 *>(prow + ((c8 ^ (r & 7)) << 4)) =
+              make_uint4(cvt_bf16x2(pv[0], pv[1]), cvt_bf16x2(pv[2], pv[3]), cvt_bf16x2(pv[4], pv[5]),
+                         cvt_bf16x2(pv[6], pv[7]));
+        }
+        fence_async_smem();
+        tc_fence_before();  // orders a rescale's TMEM stores before the next P V
+        mbar_arrive(p_full);
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-      fence_async_smem();
-      mbar_arrive(p_full);
-    }
-    if (ok && nchunks > 0) {
-      if (wait_warp(o_full, (nchunks - 1) & 1, p.status, abort_flag)) {
+      if (!ok) break;
+      // row sum over both halves (buffer by tile parity: the next write to it is two tiles away)
+      float *xs = xsum + ob * 256;
+      xs[half * 128 + r] = l;
+      if (!pair_sync()) break;
+      l += xs[(half ^ 1) * 128 + r];
+      float ov[64];
+      if (nchunks > 0) {
+        if (!wait_warp(&o_full[ob], (tl >> 1) & 1, p.status, abort_flag)) break;
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + 256 + c * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o_acc[c * 32 + e] += v[e];
-        }
+        tmem_ld32_async(tO, ov);
+        tmem_ld32_async(tO + 32, ov + 32);
+        tmem_wait_ld_regs(ov);
+        reg_fence32(ov + 32);
+        tc_fence_before();
+        mbar_arrive(&o_empty[ob]);
       } else {
-        ok = false;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) ov[e] = 0.f;
       }
-    }
-    if (ok && gi < T) {
-      const size_t row = static_cast<size_t>(hh) * T + gi;
-      if (MODE == kAttnDelta) {
-        const float mc = p.m_c[row], lc = p.l_c[row];
-        const float mc2 = mc * kLog2e;
-        const float M = fmaxf(mc2, m2);
-        const float wc = (mc == -INFINITY) ? 0.f : exp2_approx(mc2 - M);
-        const float ws = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - M);
-        const float L = lc * wc + l * ws;
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float4 *ac = reinterpret_cast<const float4 *>(p.acc_c + row * 128);
-        uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128);
+      if (gi < T) {
+        const size_t row = static_cast<size_t>(hh) * T + gi;
+        const float m2 = m_used;
+        const int d0 = half * 64;
+        if (MODE == kAttnDelta) {
+          const float mc = p.m_c[row], lc = p.l_c[row];
+          const float mc2 = mc * kLog2e;
+          const float M = fmaxf(mc2, m2);
+          const float wc = (mc == -INFINITY) ? 0.f : exp2_approx(mc2 - M);
+          const float ws = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - M);
+          const float L = lc * wc + l * ws;
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float4 *ac = reinterpret_cast<const float4 *>(p.acc_c + row * 128 + d0);
+          uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
 #pragma unroll
-        for (int e8 = 0; e8 < 16; ++e8) {
-          const float4 a0 = ac[2 * e8], a1 = ac[2 * e8 + 1];
-          const float *oa = o_acc + 8 * e8;
-          orow[e8] = make_uint4(pack_bf16x2((a0.x * wc + oa[0] * ws) * inv, (a0.y * wc + oa[1] * ws) * inv),
-                                pack_bf16x2((a0.z * wc + oa[2] * ws) * inv, (a0.w * wc + oa[3] * ws) * inv),
-                                pack_bf16x2((a1.x * wc + oa[4] * ws) * inv, (a1.y * wc + oa[5] * ws) * inv),
-                                pack_bf16x2((a1.z * wc + oa[6] * ws) * inv, (a1.w * wc + oa[7] * ws) * inv));
+          for (int e8 = 0; e8 < 8; ++e8) {
+            const float4 a0 = ac[2 * e8], a1 = ac[2 * e8 + 1];
+            const float *oa = ov + 8 * e8;
+            orow[e8] = make_uint4(cvt_bf16x2((a0.x * wc + oa[0] * ws) * inv, (a0.y * wc + oa[1] * ws) * inv),
+                                  cvt_bf16x2((a0.z * wc + oa[2] * ws) * inv, (a0.w * wc + oa[3] * ws) * inv),
+                                  cvt_bf16x2((a1.x * wc + oa[4] * ws) * inv, (a1.y * wc + oa[5] * ws) * inv),
+                                  cvt_bf16x2((a1.z * wc + oa[6] * ws) * inv, (a1.w * wc + oa[7] * ws) * inv));
+          }
+        } else if (MODE == kAttnDense) {
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
+#pragma unroll
+          for (int e8 = 0; e8 < 8; ++e8) {
+            const float *oa = ov + 8 * e8;
+            orow[e8] = make_uint4(cvt_bf16x2(oa[0] * inv, oa[1] * inv), cvt_bf16x2(oa[2] * inv, oa[3] * inv),
+                                  cvt_bf16x2(oa[4] * inv, oa[5] * inv), cvt_bf16x2(oa[6] * inv, oa[7] * inv));
+          }
+          if (half == 0) p.lse[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
+        } else {
+          if (half == 0) {
+            p.m_c[row] = (m2 == -INFINITY) ? -INFINITY : m2 * kLn2;
+            p.l_c[row] = l;
+          }
+          float4 *ac = reinterpret_cast<float4 *>(p.acc_c + row * 128 + d0);
+#pragma unroll
+          for (int e4 = 0; e4 < 16; ++e4) ac[e4] = make_float4(ov[4 * e4], ov[4 * e4 + 1], ov[4 * e4 + 2], ov[4 * e4 + 3]);
         }
-      } else if (MODE == kAttnDense) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128);
-#pragma unroll
-        for (int e8 = 0; e8 < 16; ++e8) {
-          const float *oa = o_acc + 8 * e8;
-          orow[e8] = make_uint4(pack_bf16x2(oa[0] * inv, oa[1] * inv), pack_bf16x2(oa[2] * inv, oa[3] * inv),
-                                pack_bf16x2(oa[4] * inv, oa[5] * inv), pack_bf16x2(oa[6] * inv, oa[7] * inv));
-        }
-        p.lse[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
-      } else {
-        p.m_c[row] = (m2 == -INFINITY) ? -INFINITY : m2 * kLn2;
-        p.l_c[row] = l;
-        float4 *ac = reinterpret_cast<float4 *>(p.acc_c + row * 128);
-#pragma unroll
-        for (int e4 = 0; e4 < 32; ++e4)
-          ac[e4] = make_float4(o_acc[4 * e4], o_acc[4 * e4 + 1], o_acc[4 * e4 + 2], o_acc[4 * e4 + 3]);
       }
     }
   }
@@ -478,14 +614,23 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 }
 
 template <int MODE>
+uint32_t attn_smem(int64_t T) {
+  const uint32_t mask_bytes = MODE == kAttnComplement ? ((static_cast<uint32_t>(T) + 31) / 32) * 4 : 0;
+  return 1024 + AttnCfg::kMaskOff + mask_bytes;
+}
+
+template <int MODE>
 cudaError_t launch_attn_t(const AttnParams &p, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                           cudaStream_t s) {
-  const uint32_t mask_bytes = MODE == kAttnComplement ? ((static_cast<uint32_t>(p.T) + 31) / 32) * 4 : 0;
-  const uint32_t smem = 1024 + kMaskOff + mask_bytes;
+  const uint32_t smem = attn_smem<MODE>(p.T);
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.h) * p.nb;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = static_cast<int64_t>(p.h) * p.nb;
+  const int64_t grid = std::min<int64_t>(tiles, sms);
   attn_kernel<MODE><<<static_cast<unsigned>(grid), kThreads, smem, s>>>(q, k, v, p);
   return cudaGetLastError();
 }
@@ -493,8 +638,7 @@ cudaError_t launch_attn_t(const AttnParams &p, const CUtensorMap &q, const CUten
 }  // namespace
 
 uint32_t attn_smem_bytes(int mode, int64_t T) {
-  const uint32_t mask_bytes = mode == kAttnComplement ? ((static_cast<uint32_t>(T) + 31) / 32) * 4 : 0;
-  return 1024 + kMaskOff + mask_bytes;
+  return mode == kAttnComplement ? attn_smem<kAttnComplement>(T) : attn_smem<kAttnDelta>(T);
 }
 
 cudaError_t launch_attn(int mode, const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,

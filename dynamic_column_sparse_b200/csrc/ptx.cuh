@@ -65,27 +65,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete. Bounded:
-// gives up when the CTA-wide abort flag or the device status word is set, or
-// after kWaitLimitNs, in which case it records kDevWaitTimeout in *status and
-// raises the abort flag. Returns false when it gave up.
+// gives up when the CTA-wide abort flag is set, or after about kWaitLimitNs,
+// in which case it records kDevWaitTimeout in *status and raises the abort
+// flag. Returns false when it gave up. The hot path polls only the barrier:
+// the flag and the clock are looked at every 1024 polls, so a completed phase
+// is seen at once.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
+    if ((it & 1023u) == 1023u) {
       if (*abort_flag) return false;
-      if (*(volatile int *)status != kDevOk) {
-        *abort_flag = 1;
-        return false;
-      }
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
         atomicCAS(status, kDevOk, kDevWaitTimeout);
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+
+// Barrier over `count` threads (a multiple of 32) of the CTA, id 1..15.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ----------------------------------------------------------------- TMA
@@ -178,10 +183,14 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective;
-// a warp may only touch lanes 32*(warp%4) .. 32*(warp%4)+31).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane into v, without
+// waiting: follow with tmem_wait_ld_regs(v) (and reg_fence32 for further
+// batches) before reading v (warp-collective; a warp may only touch lanes
+// 32*(warp%4) .. 32*(warp%4)+31).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float *v) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -190,9 +199,66 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  tmem_wait_ld();
+}
+
+// 32 consecutive 32-bit columns from v into this thread's TMEM lane (call
+// tmem_wait_st() before the columns are read again).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
+  const uint32_t *r = reinterpret_cast<const uint32_t *>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective;
+// a warp may only touch lanes 32*(warp%4) .. 32*(warp%4)+31).
+// The load and its wait sit in one asm statement, so no use of v can be
+// scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Waits for this thread's outstanding tcgen05.ld and ties the 32 registers of
+// v to the wait, so that no use of them moves above it.
+__device__ __forceinline__ void tmem_wait_ld_regs(float *v) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]),
+        "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+        "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Orders later uses of 32 registers after the preceding volatile asm (the
+// wait of an earlier batch of tcgen05.ld).
+__device__ __forceinline__ void reg_fence32(float *v) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
+                 "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]));
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start
@@ -229,6 +295,34 @@ __device__ __forceinline__ float exp2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for x <= 8 (used to share the exponentials of a
+// softmax between the MUFU and FMA pipes). Method: Cody-Waite style range
+// reduction x = j + f with j = round(x) by the 1.5 * 2^23 shifter (f in
+// [-1/2, 1/2]); 2^f by a degree-4 polynomial fitted for this library as a
+// near-minimax approximation of relative error on [-1/2, 1/2] (max relative
+// error 2.7e-6 in fp32); 2^j added into the exponent field. x < -125 gives 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  const float xc = fmaxf(x, -125.0f);
+  const float t = xc + 12582912.0f;
+  const float j = t - 12582912.0f;
+  const float f = xc - j;
+  float p = 9.570096619e-03f;
+  p = fmaf(p, f, 5.591785908e-02f);
+  p = fmaf(p, f, 2.402474433e-01f);
+  p = fmaf(p, f, 6.931217909e-01f);
+  p = fmaf(p, f, 9.999992847e-01f);
+  const uint32_t jb = static_cast<uint32_t>(__float_as_int(t) - 0x4B400000) << 23;
+  return x < -125.0f ? 0.0f : __uint_as_float(__float_as_uint(p) + jb);
+}
+
+// Two fp32 values to packed bf16x2 (round to nearest even) in one conversion:
+// lo in bits 0..15, hi in bits 16..31.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // GELU, tanh form: 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).
