@@ -69,8 +69,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  const int chunk = blockIdx.x % p.nchunks;
-  const int b = blockIdx.x / p.nchunks;
+  // chunk-major across blocks: index lists are ascending, so CTAs running at
+  // the same time gather W1^T rows from the same region (L2 reuse)
+  const int chunk = blockIdx.x / p.nb;
+  const int b = blockIdx.x % p.nb;
   const bool sparse = p.mode == kUpDelta;
 
   if (threadIdx.x == 0) {
@@ -264,8 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  const int slice = blockIdx.x % p.n_slices;
-  const int b = blockIdx.x / p.n_slices;
+  // slice-major across blocks: CTAs running at the same time share an N slice
+  // and sweep their (ascending) W2 rows in the same order (L2 reuse)
+  const int slice = blockIdx.x / p.nb;
+  const int b = blockIdx.x % p.nb;
   const int n0 = slice * BN;
   const int kext = DENSE ? p.krows : p.k;
   const int nk = (kext + kBK - 1) / kBK;
