@@ -19,9 +19,11 @@
 // cache (or overwrites it with result + b2 on a refresh) and writes the bf16
 // layer output.
 //
-// Warp roles: warps 0-3 = producers (thread 0 also issues the TMA tile
-// loads), warp 4 = MMA issuer and TMEM owner, warps 5-8 = epilogue (TMEM lane
-// quadrant = warp % 4).
+// Each kernel keeps two shared-memory rings: a deep one for the gathered
+// operand (filled by producer warps 0-3 with cp.async) and a shallow one for
+// the operand that arrives by tiled TMA (issued by warp 9), so that more
+// gathered bytes are in flight. Warp 4 = MMA issuer and TMEM owner, warps
+// 5-8 = epilogue (TMEM lane quadrant = warp % 4).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -30,9 +32,10 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;
 constexpr int kProducers = 128;
 constexpr int kMmaWarp = 4;
+constexpr int kTmaWarp = 9;
 constexpr int kBK = 64;  // K elements per pipeline stage = one 128-byte swizzle row
 
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
@@ -43,26 +46,33 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *s
 
 template <int BT>
 struct UpCfg {
-  static constexpr int kStages = BT == 128 ? 3 : 4;
-  static constexpr uint32_t kABytes = 128 * 128;  // 128 gathered rows x 64 bf16
-  static constexpr uint32_t kBBytes = BT * 128;   // BT tokens x 64 bf16
-  static constexpr uint32_t kBarOff = kStages * (kABytes + kBBytes);
+  static constexpr int kStagesA = BT == 128 ? 4 : 5;  // gathered W1^T rows
+  static constexpr int kStagesB = 2;                  // x tile
+  static constexpr uint32_t kABytes = 128 * 128;      // 128 gathered rows x 64 bf16
+  static constexpr uint32_t kBBytes = BT * 128;       // BT tokens x 64 bf16
+  static constexpr uint32_t kBOff = kStagesA * kABytes;
+  static constexpr uint32_t kBarOff = kBOff + kStagesB * kBBytes;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
 };
 
+// two CTAs per SM (registers capped at 65536 / (2 * kThreads)): one CTA's
+// epilogue overlaps the other's main loop
 template <int BT, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     mlp_up_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
                   const MlpUpParams p) {
   using C = UpCfg<BT>;
+  constexpr int SA = C::kStagesA, SB = C::kStagesB;
   constexpr uint32_t kIdesc = idesc_bf16(128, BT, false, false);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
-  uint8_t *sB = smem + C::kStages * C::kABytes;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-  uint64_t *empty = full + C::kStages;
-  uint64_t *acc_full = empty + C::kStages;
+  uint8_t *sB = smem + C::kBOff;
+  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+  uint64_t *a_empty = a_full + SA;
+  uint64_t *b_full = a_empty + SA;
+  uint64_t *b_empty = b_full + SB;
+  uint64_t *acc_full = b_empty + SB;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *rows = reinterpret_cast<int *>(tmem_slot + 4);
@@ -76,15 +86,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool sparse = p.mode == kUpDelta;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], DENSE ? 1 : 1 + kProducers);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&a_full[s], DENSE ? 1 : kProducers);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == kTmaWarp * 32) {
     prefetch_tmap(&tm_w1t);
     prefetch_tmap(&tm_x);
   }
@@ -113,56 +127,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = p.D / kBK;
 
   if (warp < 4) {
-    // producers: thread pt moves 16-byte chunk (pt & 7) of rows i*16 + (pt >> 3), i = 0..7
-    const int pt = threadIdx.x;
-    const uint16_t *src_row[8];
-    uint32_t dst_off[8];
+    // gathered W1^T rows: thread pt moves 16-byte chunk (pt & 7) of rows i*16 + (pt >> 3), i = 0..7
     if (!DENSE) {
+      const int pt = threadIdx.x;
+      const uint16_t *src_row[8];
+      uint32_t dst_off[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = i * 16 + (pt >> 3);
         src_row[i] = p.w1t + static_cast<size_t>(rows[r]) * p.D + (pt & 7) * 8;
         dst_off[i] = sw128_offset(r, pt & 7);
       }
-    }
-    const uint32_t a_base = smem_u32(sA);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % C::kStages;
-      const uint32_t ph = (kb / C::kStages) & 1;
-      if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
-      if (pt == 0) {
-        mbar_arrive_expect_tx(&full[s], C::kBBytes + (DENSE ? C::kABytes : 0));
-        tma_load_2d(sB + s * C::kBBytes, &tm_x, &full[s], kb * kBK, b * BT);
-        if (DENSE) tma_load_2d(sA + s * C::kABytes, &tm_w1t, &full[s], kb * kBK, chunk * 128);
-      }
-      if (!DENSE) {
+      const uint32_t a_base = smem_u32(sA);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % SA;
+        if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
         const uint32_t stage = a_base + s * C::kABytes;
 #pragma unroll
         for (int i = 0; i < 8; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
-        cp_async_arrive_noinc(&full[s]);
+        cp_async_arrive_noinc(&a_full[s]);
       }
+    }
+  } else if (warp == kTmaWarp) {
+    // x tiles (and, on a refresh, the consecutive W1^T rows) by TMA
+    for (int kb = 0; kb < nk; ++kb) {
+      if (DENSE) {
+        const int s = kb % SA;
+        if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&a_full[s], C::kABytes);
+          tma_load_2d(sA + s * C::kABytes, &tm_w1t, &a_full[s], kb * kBK, chunk * 128);
+        }
+      }
+      const int s = kb % SB;
+      if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+        tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kBK, b * BT);
+      }
+      __syncwarp();
     }
   } else if (warp == kMmaWarp) {
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % C::kStages;
-      const uint32_t ph = (kb / C::kStages) & 1;
-      if (!wait_warp(&full[s], ph, p.status, abort_flag)) {
+      const int sa = kb % SA, sb = kb % SB;
+      if (!wait_warp(&a_full[sa], (kb / SA) & 1, p.status, abort_flag) ||
+          !wait_warp(&b_full[sb], (kb / SB) & 1, p.status, abort_flag)) {
         ok = false;
         break;
       }
       if (!DENSE) fence_async_smem();
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = smem_u32(sA + s * C::kABytes);
-        const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+        const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
+        const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
           umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&a_empty[sa]);
+        umma_commit(&b_empty[sb]);
       }
       __syncwarp();
     }
@@ -238,10 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BN>
 struct DownCfg {
-  static constexpr int kStages = 4;
+  static constexpr int kStagesA = 3;                     // delta tile
+  static constexpr int kStagesB = BN == 256 ? 5 : 8;     // gathered W2 rows
   static constexpr uint32_t kABytes = 128 * 128;         // 64 K-rows x 128 tokens (two 64-token atoms)
   static constexpr uint32_t kBBytes = (BN / 64) * 8192;  // 64 K-rows x BN columns
-  static constexpr uint32_t kBarOff = kStages * (kABytes + kBBytes);
+  static constexpr uint32_t kBOff = kStagesA * kABytes;
+  static constexpr uint32_t kBarOff = kBOff + kStagesB * kBBytes;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
 };
 
@@ -250,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mlp_down_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w2,
                     const MlpDownParams p) {
   using C = DownCfg<BN>;
+  constexpr int SA = C::kStagesA, SB = C::kStagesB;
   constexpr uint32_t kIdesc = idesc_bf16(128, BN, true, true);
   constexpr uint32_t kATx = (BT / 64) * 8192;
   constexpr int kChunksPerRow = BN / 8;               // 16-byte chunks of one gathered W2 row segment
@@ -257,10 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
-  uint8_t *sB = smem + C::kStages * C::kABytes;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-  uint64_t *empty = full + C::kStages;
-  uint64_t *acc_full = empty + C::kStages;
+  uint8_t *sB = smem + C::kBOff;
+  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+  uint64_t *a_empty = a_full + SA;
+  uint64_t *b_full = a_empty + SA;
+  uint64_t *b_empty = b_full + SB;
+  uint64_t *acc_full = b_empty + SB;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -275,15 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (kext + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], DENSE ? 1 : 1 + kProducers);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&b_full[s], DENSE ? 1 : kProducers);
+      mbar_init(&b_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == kTmaWarp * 32) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_w2);
   }
@@ -293,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (BT == 64) {
     // tokens 64..127 of every A stage stay zero: the MMA always runs M = 128
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < SA; ++s) {
       uint4 *z = reinterpret_cast<uint4 *>(sA + s * C::kABytes + 8192);
       for (int i = threadIdx.x; i < 8192 / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
@@ -305,41 +340,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    // producers: warp pw gathers W2 rows pw*16 .. pw*16+15 of each 64-row stage
-    const int pt = threadIdx.x, pw = warp;
-    const int32_t *irow = DENSE ? nullptr : p.idx + static_cast<size_t>(b) * p.k;
-    const int csub = lane % kChunksPerRow;           // chunk of the row segment this lane moves
-    const int rsub = lane / kChunksPerRow;           // row within one instruction
-    const uint32_t b_base = smem_u32(sB);
-    auto load_idx = [&](int kb) -> int {             // lane < 16: index of row pw*16 + lane of stage kb
-      int c = 0;
-      if (!DENSE && lane < 16 && kb < nk) {
-        c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
-        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
-          atomicCAS(p.status, kDevOk, kDevBadIndex);
-          c = 0;
+    // gathered W2 rows: warp pw moves rows pw*16 .. pw*16+15 of each 64-row stage
+    if (!DENSE) {
+      const int pw = warp;
+      const int32_t *irow = p.idx + static_cast<size_t>(b) * p.k;
+      const int csub = lane % kChunksPerRow;           // chunk of the row segment this lane moves
+      const int rsub = lane / kChunksPerRow;           // row within one instruction
+      const uint32_t b_base = smem_u32(sB);
+      auto load_idx = [&](int kb) -> int {             // lane < 16: index of row pw*16 + lane of stage kb
+        int c = 0;
+        if (lane < 16 && kb < nk) {
+          c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
+          if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
+            atomicCAS(p.status, kDevOk, kDevBadIndex);
+            c = 0;
+          }
         }
-      }
-      return c;
-    };
-    int c_cur = load_idx(0);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % C::kStages;
-      const uint32_t ph = (kb / C::kStages) & 1;
-      const int c_next = load_idx(kb + 1);
-      if (!wait_warp(&empty[s], ph ^ 1, p.status, abort_flag)) break;
-      if (pt == 0) {
-        mbar_arrive_expect_tx(&full[s], kATx + (DENSE ? C::kBBytes : 0));
-#pragma unroll
-        for (int mt = 0; mt < BT / 64; ++mt)
-          tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &full[s], mt * 64, kb * kBK, b);
-        if (DENSE) {
-#pragma unroll
-          for (int ns = 0; ns < BN / 64; ++ns)
-            tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &full[s], n0 + ns * 64, kb * kBK);
-        }
-      }
-      if (!DENSE) {
+        return c;
+      };
+      int c_cur = load_idx(0);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % SB;
+        const int c_next = load_idx(kb + 1);
+        if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
         const uint32_t stage = b_base + s * C::kBBytes;
 #pragma unroll
         for (int i = 0; i < 16 / kRowsPerInstr; ++i) {
@@ -349,31 +372,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slab = csub >> 3, cc = csub & 7;
           cp_async_16(stage + slab * 8192 + sw128_offset(r, cc), p.w2 + static_cast<size_t>(c) * p.D + n0 + csub * 8);
         }
-        cp_async_arrive_noinc(&full[s]);
+        cp_async_arrive_noinc(&b_full[s]);
+        c_cur = c_next;
       }
-      c_cur = c_next;
+    }
+  } else if (warp == kTmaWarp) {
+    // delta / activation tiles (and, on a refresh, the consecutive W2 rows) by TMA
+    for (int kb = 0; kb < nk; ++kb) {
+      if (DENSE) {
+        const int s = kb % SB;
+        if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+#pragma unroll
+          for (int ns = 0; ns < BN / 64; ++ns)
+            tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &b_full[s], n0 + ns * 64, kb * kBK);
+        }
+      }
+      const int s = kb % SA;
+      if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&a_full[s], kATx);
+#pragma unroll
+        for (int mt = 0; mt < BT / 64; ++mt)
+          tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &a_full[s], mt * 64, kb * kBK, b);
+      }
+      __syncwarp();
     }
   } else if (warp == kMmaWarp) {
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % C::kStages;
-      const uint32_t ph = (kb / C::kStages) & 1;
-      if (!wait_warp(&full[s], ph, p.status, abort_flag)) {
+      const int sa = kb % SA, sb = kb % SB;
+      if (!wait_warp(&a_full[sa], (kb / SA) & 1, p.status, abort_flag) ||
+          !wait_warp(&b_full[sb], (kb / SB) & 1, p.status, abort_flag)) {
         ok = false;
         break;
       }
       if (!DENSE) fence_async_smem();
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = smem_u32(sA + s * C::kABytes);
-        const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+        const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
+        const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 8192, 1024);
           const uint64_t bd = sdesc_sw128(b0 + kk * 2048, 8192, 1024);
           umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&a_empty[sa]);
+        umma_commit(&b_empty[sb]);
       }
       __syncwarp();
     }
