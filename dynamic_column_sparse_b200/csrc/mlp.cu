@@ -273,6 +273,10 @@ struct DownCfg {
   static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
 };
 
+// Persistent: CTA c handles tiles c, c + gridDim.x, ...; the two TMEM
+// accumulators alternate between tiles so the epilogue of one tile overlaps
+// the main loop of the next. Ring stages and their parities follow one
+// running k-step counter across tiles.
 template <int BT, int BN, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 1)
     mlp_down_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w2,
@@ -291,17 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *a_empty = a_full + SA;
   uint64_t *b_full = a_empty + SA;
   uint64_t *b_empty = b_full + SB;
-  uint64_t *acc_full = b_empty + SB;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  uint64_t *acc_full = b_empty + SB;   // [2]
+  uint64_t *acc_empty = acc_full + 2;  // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  // slice-major across blocks: CTAs running at the same time share an N slice
-  // and sweep their (ascending) W2 rows in the same order (L2 reuse)
-  const int slice = blockIdx.x / p.nb;
-  const int b = blockIdx.x % p.nb;
-  const int n0 = slice * BN;
+  const int ntiles = p.nb * p.n_slices;
   const int kext = DENSE ? p.krows : p.k;
   const int nk = (kext + kBK - 1) / kBK;
 
@@ -314,7 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b_full[s], DENSE ? 1 : kProducers);
       mbar_init(&b_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -323,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_w2);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   if (BT == 64) {
@@ -339,104 +343,141 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // slice-major across blocks: CTAs running at the same time share an N slice
+  // and sweep their (ascending) W2 rows in the same order (L2 reuse)
   if (warp < 4) {
     // gathered W2 rows: warp pw moves rows pw*16 .. pw*16+15 of each 64-row stage
     if (!DENSE) {
       const int pw = warp;
-      const int32_t *irow = p.idx + static_cast<size_t>(b) * p.k;
       const int csub = lane % kChunksPerRow;           // chunk of the row segment this lane moves
       const int rsub = lane / kChunksPerRow;           // row within one instruction
       const uint32_t b_base = smem_u32(sB);
-      auto load_idx = [&](int kb) -> int {             // lane < 16: index of row pw*16 + lane of stage kb
-        int c = 0;
-        if (lane < 16 && kb < nk) {
-          c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
-          if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
-            atomicCAS(p.status, kDevOk, kDevBadIndex);
-            c = 0;
+      int kg = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
+        const int32_t *irow = p.idx + static_cast<size_t>(b) * p.k;
+        auto load_idx = [&](int kb) -> int {           // lane < 16: index of row pw*16 + lane of stage kb
+          int c = 0;
+          if (lane < 16 && kb < nk) {
+            c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
+            if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
+              atomicCAS(p.status, kDevOk, kDevBadIndex);
+              c = 0;
+            }
           }
-        }
-        return c;
-      };
-      int c_cur = load_idx(0);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % SB;
-        const int c_next = load_idx(kb + 1);
-        if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
-        const uint32_t stage = b_base + s * C::kBBytes;
+          return c;
+        };
+        int c_cur = load_idx(0);
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % SB;
+          const int c_next = load_idx(kb + 1);
+          if (!wait_warp(&b_empty[s], ((kg / SB) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t stage = b_base + s * C::kBBytes;
 #pragma unroll
-        for (int i = 0; i < 16 / kRowsPerInstr; ++i) {
-          const int rr = i * kRowsPerInstr + rsub;   // 0..15 within this warp's rows
-          const int r = pw * 16 + rr;                // row of the stage
-          const int c = __shfl_sync(0xffffffffu, c_cur, rr);
-          const int slab = csub >> 3, cc = csub & 7;
-          cp_async_16(stage + slab * 8192 + sw128_offset(r, cc), p.w2 + static_cast<size_t>(c) * p.D + n0 + csub * 8);
+          for (int i = 0; i < 16 / kRowsPerInstr; ++i) {
+            const int rr = i * kRowsPerInstr + rsub;   // 0..15 within this warp's rows
+            const int r = pw * 16 + rr;                // row of the stage
+            const int c = __shfl_sync(0xffffffffu, c_cur, rr);
+            const int slab = csub >> 3, cc = csub & 7;
+            cp_async_16(stage + slab * 8192 + sw128_offset(r, cc),
+                        p.w2 + static_cast<size_t>(c) * p.D + n0 + csub * 8);
+          }
+          cp_async_arrive_noinc(&b_full[s]);
+          c_cur = c_next;
         }
-        cp_async_arrive_noinc(&b_full[s]);
-        c_cur = c_next;
       }
     }
   } else if (warp == kTmaWarp) {
     // delta / activation tiles (and, on a refresh, the consecutive W2 rows) by TMA
-    for (int kb = 0; kb < nk; ++kb) {
-      if (DENSE) {
-        const int s = kb % SB;
-        if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+    int kg = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        if (DENSE) {
+          const int s = kg % SB;
+          if (!wait_warp(&b_empty[s], ((kg / SB) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
 #pragma unroll
-          for (int ns = 0; ns < BN / 64; ++ns)
-            tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &b_full[s], n0 + ns * 64, kb * kBK);
+            for (int ns = 0; ns < BN / 64; ++ns)
+              tma_load_2d(sB + s * C::kBBytes + ns * 8192, &tm_w2, &b_full[s], n0 + ns * 64, kb * kBK);
+          }
         }
-      }
-      const int s = kb % SA;
-      if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&a_full[s], kATx);
+        const int s = kg % SA;
+        if (!wait_warp(&a_empty[s], ((kg / SA) & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&a_full[s], kATx);
 #pragma unroll
-        for (int mt = 0; mt < BT / 64; ++mt)
-          tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &a_full[s], mt * 64, kb * kBK, b);
+          for (int mt = 0; mt < BT / 64; ++mt)
+            tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &a_full[s], mt * 64, kb * kBK, b);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
   } else if (warp == kMmaWarp) {
+    int kg = 0, tl = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int sa = kb % SA, sb = kb % SB;
-      if (!wait_warp(&a_full[sa], (kb / SA) & 1, p.status, abort_flag) ||
-          !wait_warp(&b_full[sb], (kb / SB) & 1, p.status, abort_flag)) {
-        ok = false;
-        break;
-      }
-      if (!DENSE) fence_async_smem();
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
+      const int ab = tl & 1;
+      const uint32_t tacc = tmem + ab * BN;
+      if (!wait_warp(&acc_empty[ab], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
-        const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 8192, 1024);
-          const uint64_t bd = sdesc_sw128(b0 + kk * 2048, 8192, 1024);
-          umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int sa = kg % SA, sb = kg % SB;
+        if (!wait_warp(&a_full[sa], (kg / SA) & 1, p.status, abort_flag) ||
+            !wait_warp(&b_full[sb], (kg / SB) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
         }
-        umma_commit(&a_empty[sa]);
-        umma_commit(&b_empty[sb]);
+        if (!DENSE) fence_async_smem();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 8192, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, 8192, 1024);
+            umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+          }
+          umma_commit(&a_empty[sa]);
+          umma_commit(&b_empty[sb]);
+        }
+        __syncwarp();
       }
+      if (ok && lane == 0) umma_commit(&acc_full[ab]);
       __syncwarp();
     }
-    if (ok && lane == 0) umma_commit(acc_full);
-    __syncwarp();
   } else {
     const int q = warp & 3;
     const int t = q * 32 + lane;
-    const int64_t grow = static_cast<int64_t>(b) * BT + t;
-    const bool valid = t < BT && grow < p.T;
-    if (wait_warp(acc_full, 0, p.status, abort_flag)) {
+    int tl = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+      const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
+      const int ab = tl & 1;
+      const int64_t grow = static_cast<int64_t>(b) * BT + t;
+      const bool valid = t < BT && grow < p.T;
+      if (!wait_warp(&acc_full[ab], (tl >> 1) & 1, p.status, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int nc = 0; nc < BN / 32; ++nc) {
         float acc[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + nc * 32, acc);
+        tmem_ld32(tmem + ab * BN + (static_cast<uint32_t>(q * 32) << 16) + nc * 32, acc);
+        if (nc == BN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
+        }
         if (valid) {
           const int n = n0 + nc * 32;
           float4 *y4 = reinterpret_cast<float4 *>(p.y_cache + grow * p.D + n);
@@ -460,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *o4 = reinterpret_cast<uint4 *>(p.out + grow * p.D + n);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              o4[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]), pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
-                                 pack_bf16x2(y[8 * v + 4], y[8 * v + 5]), pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+              o4[v] = make_uint4(cvt_bf16x2(y[8 * v], y[8 * v + 1]), cvt_bf16x2(y[8 * v + 2], y[8 * v + 3]),
+                                 cvt_bf16x2(y[8 * v + 4], y[8 * v + 5]), cvt_bf16x2(y[8 * v + 6], y[8 * v + 7]));
           }
         }
       }
@@ -470,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, BN);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 2 * BN);
 }
 
 // out = bf16(y) when a sparse step selects nothing
@@ -502,7 +543,10 @@ cudaError_t launch_down_t(const MlpDownParams &p, const CUtensorMap &a, const CU
   using C = DownCfg<BN>;
   cudaError_t e = set_smem(mlp_down_kernel<BT, BN, DENSE>, C::kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.nb) * p.n_slices;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.n_slices, sms);
   mlp_down_kernel<BT, BN, DENSE><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(a, w, p);
   return cudaGetLastError();
 }
