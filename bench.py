@@ -58,6 +58,22 @@ def flops_step(w):
     return up, down, attn
 
 
+def max_over_ranks(x, device=None):
+    """Maximum of a per-rank float over all ranks of the default process group (x when there is none)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_us_per_layer(ms_step_max, world):
+    """Whole-job microseconds per layer-step: every rank processes one layer per step (weak scaling)."""
+    return ms_step_max * 1e3 / world
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -305,13 +321,6 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     from dynamic_column_sparse_b200 import chipmunk as cm
     cm.load_library()
     w = dict(W)
@@ -358,7 +367,7 @@ def run_gpu(args):
     t_up = [e[0].elapsed_time(e[1]) for e in evs]
     t_down = [e[1].elapsed_time(e[2]) for e in evs]
     t_attn = [e[2].elapsed_time(e[3]) for e in evs]
-    ms_step = max_over_ranks(statistics.mean(tot))
+    ms_step = max_over_ranks(statistics.mean(tot), dev)
     status = cm.read_device_status()
     assert status == 0, f"device status {status}"
 
@@ -394,7 +403,7 @@ def run_gpu(args):
         b.synchronize()
         e2e_ts.append(a.elapsed_time(b))
     barrier()
-    e2e_ms = max_over_ranks(statistics.mean(e2e_ts))
+    e2e_ms = max_over_ranks(statistics.mean(e2e_ts), dev)
     h2d = x_d.numel() * 2 + sum(t.numel() * 2 for t in qkv_d)
     d2h = out_h.numel() * 2 + o_h.numel() * 2
 
@@ -414,7 +423,7 @@ def run_gpu(args):
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "traffic": tr, "peak_source": f"{peak_src} bf16 dense (burst)"}
 
-    us_layer = ms_step * 1e3 / world
+    us_layer = job_us_per_layer(ms_step, world)
     res = {
         "metric": METRIC, "value": round(us_layer, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
@@ -428,7 +437,7 @@ def run_gpu(args):
         "useful_tflops": round(flops * world / (ms_step * 1e-3) / 1e12, 1),
         "pct_bf16_peak": round(100 * flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 2),
         "kernels": kern, "roofline": roofline,
-        "e2e": {"value": round(e2e_ms * 1e3 / world, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        "e2e": {"value": round(job_us_per_layer(e2e_ms, world), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,

@@ -36,6 +36,7 @@ EXPORTS = (
     "chipmunk_attn_delta", "chipmunk_dense_refresh",
     "chipmunk_gather_cols", "chipmunk_scatter_cols", "chipmunk_workspace_bytes", "chipmunk_status_string",
     "chipmunk_last_error", "chipmunk_read_device_status", "chipmunk_version", "chipmunk_mlp_delta_noalloc",
+    "chipmunk_selftest_bounded_wait",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -98,6 +99,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "chipmunk_scatter_cols": [vp, i64, i64, i32, vp, i32, vp, vp],
             "chipmunk_read_device_status": [ctypes.POINTER(i32), vp],
             "chipmunk_mlp_delta_noalloc": [ctypes.POINTER(MlpArgs), vp],
+            "chipmunk_selftest_bounded_wait": [vp],
         }
         for name, argtypes in sig.items():
             fn = getattr(lib, name)

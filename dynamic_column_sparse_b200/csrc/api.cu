@@ -180,8 +180,8 @@ size_t mlp_delta_ws(const chipmunk_mlp_args *a) {
 }
 
 chipmunk_status topk_impl(const float *scores, int64_t rows, int64_t n, int64_t ld_scores, int32_t k, int32_t *idx,
-                          int64_t ld_idx, cudaStream_t s) {
-  cm::TopkParams p{scores, rows, n, ld_scores, k, idx, ld_idx};
+                          int64_t ld_idx, int *status, cudaStream_t s) {
+  cm::TopkParams p{scores, rows, n, ld_scores, k, idx, ld_idx, status};
   CM_CUDA(cm::launch_topk(p, s), "top-k launch");
   return CHIPMUNK_OK;
 }
@@ -275,7 +275,7 @@ chipmunk_status chipmunk_topk_cols(const float *scores, int64_t rows, int64_t n,
   if (!aligned16(scores) || !aligned16(idx)) return fail(CHIPMUNK_ERR_ALIGNMENT, "scores or idx not 16-byte aligned");
   int *status = nullptr;
   CM_CHECK(device_setup(&status));
-  return topk_impl(scores, rows, n, ld_scores, k, idx, ld_idx, static_cast<cudaStream_t>(stream));
+  return topk_impl(scores, rows, n, ld_scores, k, idx, ld_idx, status, static_cast<cudaStream_t>(stream));
 }
 
 chipmunk_status chipmunk_mlp_delta(const chipmunk_mlp_args *a, void *ws, size_t ws_bytes, chipmunk_stream stream) {
@@ -347,7 +347,7 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
                          cm::kDownOverwrite, static_cast<const uint16_t *>(a->w2), int(a->H), nullptr,
                          static_cast<const uint16_t *>(a->b2), a->y_cache, static_cast<uint16_t *>(a->out), status};
     CM_CUDA(cm::launch_mlp_down(dp, tm_a, tm_w2, true, s), "MLP refresh down-projection launch");
-    return topk_impl(r->scores, nb, a->H, a->H, a->k, a->idx, a->k, s);
+    return topk_impl(r->scores, nb, a->H, a->H, a->k, a->idx, a->k, status, s);
   }
   if (r->kind == CHIPMUNK_REFRESH_ATTN) {
     const chipmunk_attn_args *a = &r->attn;
@@ -372,7 +372,7 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
     CM_CUDA(cm::launch_attn(cm::kAttnDense, dense, tm_q, tm_k, tm_v, s), "attention refresh dense launch");
     cm::MassParams mp{int(a->T), a->h, int(nb), sl2, lse, r->scores, status};
     CM_CUDA(cm::launch_attn_mass(mp, tm_q, tm_k, s), "attention mass launch");
-    CM_CHECK(topk_impl(r->scores, int64_t(a->h) * nb, a->T, a->T, a->k, a->idx, a->k, s));
+    CM_CHECK(topk_impl(r->scores, int64_t(a->h) * nb, a->T, a->T, a->k, a->idx, a->k, status, s));
     CM_CUDA(cm::launch_attn(cm::kAttnComplement, dense, tm_q, tm_k, tm_v, s), "attention complement launch");
     return CHIPMUNK_OK;
   }
@@ -390,7 +390,7 @@ chipmunk_status chipmunk_gather_cols(const void *a_cache, int64_t nb, int64_t H,
   int *status = nullptr;
   CM_CHECK(device_setup(&status));
   CM_CUDA(cm::launch_gather_cols(static_cast<const uint16_t *>(a_cache), nb, H, Bt, idx, k,
-                                 static_cast<uint16_t *>(packed), static_cast<cudaStream_t>(stream)),
+                                 static_cast<uint16_t *>(packed), status, static_cast<cudaStream_t>(stream)),
           "gather launch");
   return CHIPMUNK_OK;
 }
@@ -406,7 +406,7 @@ chipmunk_status chipmunk_scatter_cols(const void *packed, int64_t nb, int64_t H,
   int *status = nullptr;
   CM_CHECK(device_setup(&status));
   CM_CUDA(cm::launch_scatter_cols(static_cast<const uint16_t *>(packed), nb, H, Bt, idx, k,
-                                  static_cast<uint16_t *>(a_cache), static_cast<cudaStream_t>(stream)),
+                                  static_cast<uint16_t *>(a_cache), status, static_cast<cudaStream_t>(stream)),
           "scatter launch");
   return CHIPMUNK_OK;
 }
@@ -453,6 +453,13 @@ chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args *a, chipmunk_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CM_CHECK(mlp_up_impl(a, ws, status, s));
   return mlp_down_impl(a, ws, status, s);
+}
+
+chipmunk_status chipmunk_selftest_bounded_wait(chipmunk_stream stream) {
+  int *status = nullptr;
+  CM_CHECK(device_setup(&status));
+  CM_CUDA(cm::launch_selftest_wait(status, static_cast<cudaStream_t>(stream)), "self-test launch");
+  return CHIPMUNK_OK;
 }
 
 chipmunk_status chipmunk_read_device_status(int32_t *host_out, chipmunk_stream stream) {

@@ -15,15 +15,16 @@ struct TopkParams {
   int32_t k;
   int32_t *idx;
   int64_t ld_idx;
+  int *status;
 };
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
 
 // ------------------------------------------------------------------ cache column gather / scatter
 
 cudaError_t launch_gather_cols(const uint16_t *a_cache, int64_t nb, int64_t H, int Bt, const int32_t *idx, int k,
-                               uint16_t *packed, cudaStream_t s);
+                               uint16_t *packed, int *status, cudaStream_t s);
 cudaError_t launch_scatter_cols(const uint16_t *packed, int64_t nb, int64_t H, int Bt, const int32_t *idx, int k,
-                                uint16_t *a_cache, cudaStream_t s);
+                                uint16_t *a_cache, int *status, cudaStream_t s);
 
 // ------------------------------------------------------------------ MLP
 
@@ -90,6 +91,9 @@ struct MassParams {
   float *mass;            // [h][nb][T]
   int *status;
 };
+// One CTA waiting on a barrier nothing signals (bounded: records a timeout).
+cudaError_t launch_selftest_wait(int *status, cudaStream_t s);
+
 cudaError_t launch_attn_mass(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k, cudaStream_t s);
 
 }  // namespace cm

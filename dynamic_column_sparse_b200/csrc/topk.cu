@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams p) {
   const int tid = threadIdx.x;
   const int n = static_cast<int>(p.n);
   const int k = p.k;
+  if (*(volatile int *)p.status != kDevOk) return;  // an earlier failure is pending: do nothing
 
   for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
     const float *src = p.scores + row * p.ld_scores;

@@ -67,11 +67,74 @@ def raw_bits(seed: int, tensor_id: int, start: int, count: int) -> np.ndarray:
         return _mix(key + n * GOLDEN)
 
 
+_CHUNK = 1 << 20
+
+
+def _normal_chunk(key: np.uint64, start: int, count: int, out: np.ndarray) -> None:
+    z = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z *= GOLDEN
+        z += key
+        t = np.empty_like(z)
+        np.right_shift(z, np.uint64(30), out=t)
+        z ^= t
+        z *= _C1
+        np.right_shift(z, np.uint64(27), out=t)
+        z ^= t
+        z *= _C2
+        np.right_shift(z, np.uint64(31), out=t)
+        z ^= t
+    m16 = np.uint64(0xFFFF)
+    np.bitwise_and(z, m16, out=t)
+    s = t.copy()
+    for sh in (16, 32):
+        np.right_shift(z, np.uint64(sh), out=t)
+        t &= m16
+        s += t
+    np.right_shift(z, np.uint64(48), out=t)
+    s += t
+    np.multiply(s.astype(np.float64) + 2.0, 1.0 / 65536.0, out=out)
+    out -= 2.0
+    out *= SQRT3
+
+
 def normal_f64(seed: int, tensor_id: int, count: int, start: int = 0) -> np.ndarray:
-    bits = raw_bits(seed, tensor_id, start, count)
+    """Irwin-Hall(4) normals of stream (seed, tensor_id), draws start .. start+count-1."""
+    key = stream_key(seed, tensor_id)
+    out = np.empty(count, dtype=np.float64)
+    for c0 in range(0, count, _CHUNK):
+        n = min(_CHUNK, count - c0)
+        _normal_chunk(key, start + c0, n, out[c0:c0 + n])
+    return out
+
+
+def normal_f64_at(seed: int, tensor_id: int, counters: np.ndarray) -> np.ndarray:
+    """The normals of stream (seed, tensor_id) at arbitrary draw numbers
+    (the same values normal_f64 gives at those positions)."""
+    key = stream_key(seed, tensor_id)
+    cnt = np.asarray(counters, dtype=np.uint64).ravel()
+    bits = np.empty(cnt.size, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        for c0 in range(0, cnt.size, _CHUNK):
+            bits[c0:c0 + _CHUNK] = _mix(key + (cnt[c0:c0 + _CHUNK] + np.uint64(1)) * GOLDEN)
     m16 = np.uint64(0xFFFF)
     s = (bits & m16) + ((bits >> np.uint64(16)) & m16) + ((bits >> np.uint64(32)) & m16) + (bits >> np.uint64(48))
-    return ((s.astype(np.float64) + 2.0) / 65536.0 - 2.0) * SQRT3
+    return (((s.astype(np.float64) + 2.0) / 65536.0 - 2.0) * SQRT3).reshape(np.shape(counters))
+
+
+def rows_bf16(seed: int, tensor_id: int, row_len: int, rows: np.ndarray, std: float = 1.0) -> np.ndarray:
+    """Selected rows of the row-major tensor normal_bf16(seed, tensor_id, (R, row_len), std)."""
+    rows = np.asarray(rows, dtype=np.uint64)
+    counters = rows[:, None] * np.uint64(row_len) + np.arange(row_len, dtype=np.uint64)[None, :]
+    return to_bf16(std * normal_f64_at(seed, tensor_id, counters))
+
+
+def drift_rows_bf16(prev_rows_bits: np.ndarray, seed: int, tensor_id: int, row_len: int, rows: np.ndarray,
+                    sigma: float) -> np.ndarray:
+    """drift_bf16 restricted to selected rows of a row-major tensor."""
+    rows = np.asarray(rows, dtype=np.uint64)
+    counters = rows[:, None] * np.uint64(row_len) + np.arange(row_len, dtype=np.uint64)[None, :]
+    return to_bf16(bf16_bits_to_f64(prev_rows_bits) + sigma * normal_f64_at(seed, tensor_id, counters))
 
 
 def uniform_f64(seed: int, tensor_id: int, count: int, start: int = 0) -> np.ndarray:

@@ -276,6 +276,17 @@ CHIPMUNK_API const char *chipmunk_last_error(void);
  */
 CHIPMUNK_API chipmunk_status chipmunk_read_device_status(int32_t *host_out, chipmunk_stream stream);
 
+/*
+ * Diagnostic for failure detection (no counterpart in the post): launches one
+ * CTA that waits, with the same bounded wait every kernel uses, on a barrier
+ * nothing signals. The wait gives up after about 2 s and records
+ * CHIPMUNK_DEV_WAIT_TIMEOUT in the device status word; the kernel then
+ * returns normally (no trap, no fault) and the context stays usable. Read
+ * and clear the word with chipmunk_read_device_status. Kernels launched
+ * while the word is set return at entry without doing work.
+ */
+CHIPMUNK_API chipmunk_status chipmunk_selftest_bounded_wait(chipmunk_stream stream);
+
 /* Library version, e.g. "0.1.0". */
 CHIPMUNK_API const char *chipmunk_version(void);
 

@@ -244,6 +244,15 @@ def dense_attention(q, k, v, scale):
     return O, lse
 
 
+def attn_mass_rows(q_rows, k, scale):
+    """Attention mass of each key for one query block ``q_rows`` [n][d] over keys ``k`` [m][d]:
+    the column sums of the row softmax, ``sum over i of softmax_i(j)``."""
+    s = scale * (q_rows @ k.T)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p.sum(axis=0)
+
+
 def attn_mass(q, k, scale, Bt):
     """Attention mass of each key for each query block: column sums of the softmax.
 
@@ -254,10 +263,7 @@ def attn_mass(q, k, scale, Bt):
     out = np.zeros((h, nb, T))
     for hh in range(h):
         for b, r0, r1 in blocks(T, Bt):
-            s = scale * (q[hh, r0:r1] @ k[hh].T)
-            p = np.exp(s - s.max(axis=1, keepdims=True))
-            p /= p.sum(axis=1, keepdims=True)
-            out[hh, b] = p.sum(axis=0)
+            out[hh, b] = attn_mass_rows(q[hh, r0:r1], k[hh], scale)
     return out
 
 

@@ -1,0 +1,99 @@
+"""Multi-step loop: dense refresh on steps 0 and 5 of 10, sparse steps between,
+inputs drifting each step (x_{s+1} = x_s + 0.03 N(0,1)).
+
+The GPU chain (SparseDeltaMLP / SparseDeltaAttention over the C ABI) and the
+oracle chain (fp64 caches, its own selections) run the same schedule from the
+same inputs; every step's outputs must agree within the parity bar. The
+chains select independently, so a near-tie may pick a different column on
+each side; the bar absorbs that. The gap to a fully dense fp64 run (the
+method's own approximation error) is printed for information.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from dynamic_column_sparse_b200 import synth
+from helpers import assert_parity, dev_bf16, f64_of_bf16, heads_first
+
+pytestmark = pytest.mark.gpu
+
+DENSE_STEPS = (0, 5)
+STEPS = 10
+
+
+def drift_chain(first_bits, seed, tid, sigma, steps):
+    xs = [first_bits]
+    for s in range(1, steps):
+        xs.append(synth.drift_bf16(xs[-1], seed + 1000 * s, tid, sigma))
+    return xs
+
+
+def run_mlp_loop(T, D, H, permille, seed=3):
+    import torch
+    from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaMLP
+    w1t = synth.normal_bf16(seed, synth.TID["w1t"], (H, D), std=1 / math.sqrt(D))
+    b1 = synth.normal_bf16(seed, synth.TID["b1"], (H,), std=0.02)
+    w2 = synth.normal_bf16(seed, synth.TID["w2"], (H, D), std=1 / math.sqrt(H))
+    b2 = synth.normal_bf16(seed, synth.TID["b2"], (D,), std=0.02)
+    xs = drift_chain(synth.normal_bf16(seed, synth.TID["x_prev"], (T, D)), seed, synth.TID["x_drift"], 0.03, STEPS)
+    W1 = np.ascontiguousarray(O.bf16_decode(w1t).T)
+    B1, W2, B2 = O.bf16_decode(b1), O.bf16_decode(w2), O.bf16_decode(b2)
+    layer = SparseDeltaMLP(dev_bf16(w1t), dev_bf16(b1), dev_bf16(w2), dev_bf16(b2), T, 128, permille)
+    sched = Schedule(DENSE_STEPS)
+    k = O.k_from_density(H, permille)
+    A = Y = idx = None
+    worst = 0.0
+    for s in range(STEPS):
+        out = f64_of_bf16(sched.run(layer, s, dev_bf16(xs[s])))
+        x = O.bf16_decode(xs[s])
+        if sched.is_dense(s):
+            r = O.mlp_refresh(x, W1, B1, W2, B2, A, 128, k, first_step=A is None)
+            A, Y, idx = r["a"], r["y"], r["idx"]
+        else:
+            A, Y = O.mlp_delta(x, W1, B1, W2, idx, A, Y, 128)
+        ratio, _ = assert_parity(out, Y, f"MLP output, step {s}", bf16_out=True)
+        _, dense = O.dense_mlp(x, W1, B1, W2, B2)
+        gap = float(np.sqrt(np.mean((Y - dense) ** 2) / np.mean(dense ** 2)))
+        worst = max(worst, ratio)
+        print(f"mlp step {s}: max|err|/rms {ratio:.4f}  method gap to dense {gap:.4f}")
+    torch.cuda.synchronize()
+    return worst
+
+
+def run_attn_loop(T, h, permille, seed=4):
+    import torch
+    from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaAttention
+    chains = {n: drift_chain(synth.normal_bf16(seed, synth.TID[n + "_prev"], (T, h, 128)), seed,
+                             synth.TID[n + "_drift"], 0.03, STEPS) for n in ("q", "k", "v")}
+    layer = SparseDeltaAttention(T, h, "cuda", permille)
+    sched = Schedule(DENSE_STEPS)
+    scale = 1.0 / math.sqrt(128)
+    kk = O.k_from_density(T, permille)
+    cache = None
+    for s in range(STEPS):
+        out = heads_first(f64_of_bf16(sched.run(layer, s, *(dev_bf16(chains[n][s]) for n in ("q", "k", "v")))))
+        q, k, v = (np.ascontiguousarray(O.bf16_decode(chains[n][s]).transpose(1, 0, 2)) for n in ("q", "k", "v"))
+        if sched.is_dense(s):
+            r = O.attn_refresh(q, k, v, scale, 128, kk)
+            cache, ref = (r["idx"], r["m_c"], r["l_c"], r["acc_c"]), r["O"]
+        else:
+            ref = O.attn_delta(q, k, v, *cache, scale, 128)
+        ratio, _ = assert_parity(out, ref, f"attention output, step {s}", bf16_out=True)
+        print(f"attn step {s}: max|err|/rms {ratio:.4f}")
+    torch.cuda.synchronize()
+
+
+def test_loop_flux_shape_mlp():
+    run_mlp_loop(4352, 3072, 12288, 300)
+
+
+def test_loop_flux_shape_attention():
+    run_attn_loop(4352, 24, 165)
+
+
+@pytest.mark.parametrize("permille", [500, 300, 150, 70])  # 50 / 70 / 85 / 93 % sparse
+def test_loop_sparsity_sweep(permille):
+    run_mlp_loop(1024, 512, 2048, permille)
+    run_attn_loop(1024, 4, permille)

@@ -1,0 +1,182 @@
+"""Mistakes planted in the oracle must be caught by its pins.
+
+Each mutation replaces one oracle function with a copy carrying a plausible
+error (a dropped term, a wrong sign or index, a transposed reduction, a wrong
+tie rule, a missing scale). The pin suite in test_oracle_pins.py is then run
+against the mutated oracle; at least one pin must fail. Everything runs on
+the CPU.
+"""
+import inspect
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.chipmunk_oracle as OC
+import test_oracle_pins as pins
+
+ORIG = {name: getattr(OC, name) for name in ("mlp_delta", "attn_partial")}
+
+
+def _all_pins():
+    calls = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if params:
+            argnames = [a.strip() for a in params[0].args[0].split(",")]
+            for values in params[0].args[1]:
+                calls.append((name, fn, dict(zip(argnames, values))))
+        else:
+            calls.append((name, fn, {}))
+    return calls
+
+
+def _caught(monkeypatch, fname, mutant):
+    monkeypatch.setattr(OC, fname, mutant)
+    monkeypatch.setattr(oracle, fname, mutant)
+    failed = []
+    for name, fn, kwargs in _all_pins():
+        try:
+            fn(**kwargs)
+        except AssertionError:
+            failed.append(name)
+    return failed
+
+
+def _gelu_no_cubic(u):
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * u))
+
+
+def _gelu_sign(u):
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1.0 - np.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+
+
+def _mlp_delta_sign(x, W1, b1, W2, idx, A_cache, Y_cache, Bt):
+    A_new, Y_new = np.array(A_cache, dtype=float), np.array(Y_cache, dtype=float)
+    for b, r0, r1 in OC.blocks(x.shape[0], Bt):
+        S = np.asarray(idx[b], dtype=np.int64)
+        if S.size:
+            a = OC.gelu_tanh(x[r0:r1] @ W1[:, S] + b1[S])
+            Y_new[r0:r1] += (A_cache[r0:r1][:, S] - a) @ W2[S, :]
+            A_new[r0:r1, S] = a
+    return A_new, Y_new
+
+
+def _mlp_delta_no_bias(x, W1, b1, W2, idx, A_cache, Y_cache, Bt):
+    return ORIG["mlp_delta"](x, W1, np.zeros_like(b1), W2, idx, A_cache, Y_cache, Bt)
+
+
+def _mlp_delta_stale_cache(x, W1, b1, W2, idx, A_cache, Y_cache, Bt):
+    _, Y_new = ORIG["mlp_delta"](x, W1, b1, W2, idx, A_cache, Y_cache, Bt)
+    return np.array(A_cache, dtype=float), Y_new
+
+
+def _topk_high_ties(scores32, k):
+    scores32 = np.atleast_2d(np.asarray(scores32, dtype=np.float32))
+    keys = OC.ordered_key(scores32).astype(np.int64)
+    out = np.empty((scores32.shape[0], k), dtype=np.int32)
+    for r in range(scores32.shape[0]):
+        n = scores32.shape[1]
+        order = n - 1 - np.argsort(-keys[r][::-1], kind="stable")
+        out[r] = np.sort(order[:k])
+    return out
+
+
+def _topk_unsorted(scores32, k):
+    scores32 = np.atleast_2d(np.asarray(scores32, dtype=np.float32))
+    keys = OC.ordered_key(scores32).astype(np.int64)
+    out = np.empty((scores32.shape[0], k), dtype=np.int32)
+    for r in range(scores32.shape[0]):
+        out[r] = np.argsort(-keys[r], kind="stable")[:k]
+    return out
+
+
+def _key_no_neg_zero(s32):
+    bits = np.ascontiguousarray(s32, dtype=np.float32).view(np.uint32).copy()
+    neg = (bits & np.uint32(0x80000000)) != 0
+    return np.where(neg, ~bits, bits | np.uint32(0x80000000)).astype(np.uint32)
+
+
+def _merge_wrong_weight(p1, p2):
+    m1, l1, a1 = p1
+    m2, l2, a2 = p2
+    M = np.maximum(m1, m2)
+    with np.errstate(invalid="ignore", over="ignore"):
+        w1 = np.where(m1 == -np.inf, 0.0, np.exp(M - m1))
+        w2 = np.where(m2 == -np.inf, 0.0, np.exp(M - m2))
+    return M, l1 * w1 + l2 * w2, a1 * w1[:, None] + a2 * w2[:, None]
+
+
+def _partial_no_scale(q, k, v, scale):
+    return ORIG["attn_partial"](q, k, v, 1.0)
+
+
+def _mass_wrong_axis(q, k, scale, Bt):
+    h, T, d = q.shape
+    nb = (T + Bt - 1) // Bt
+    out = np.zeros((h, nb, T))
+    for hh in range(h):
+        for b, r0, r1 in OC.blocks(T, Bt):
+            s = scale * (q[hh, r0:r1] @ k[hh].T)
+            p = np.exp(s - s.max(axis=0, keepdims=True))
+            p /= p.sum(axis=0, keepdims=True)
+            out[hh, b] = p.sum(axis=0)
+    return out
+
+
+def _complement_keeps_selected(q, k, v, idx, scale, Bt):
+    h, T, d = q.shape
+    m_c, l_c, acc_c = np.full((h, T), -np.inf), np.zeros((h, T)), np.zeros((h, T, d))
+    for hh in range(h):
+        for b, r0, r1 in OC.blocks(T, Bt):
+            m_c[hh, r0:r1], l_c[hh, r0:r1], acc_c[hh, r0:r1] = OC.attn_partial(q[hh, r0:r1], k[hh], v[hh], scale)
+    return m_c, l_c, acc_c
+
+
+def _scores_no_abs(a, A_cache, Bt, first_step):
+    T, H = a.shape
+    out = np.zeros(((T + Bt - 1) // Bt, H))
+    for b, r0, r1 in OC.blocks(T, Bt):
+        d = a[r0:r1] if first_step else a[r0:r1] - A_cache[r0:r1]
+        out[b] = d.sum(axis=0)
+    return out
+
+
+def _bf16_truncate(x):
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+MUTATIONS = {
+    "gelu_tanh: cubic term dropped": ("gelu_tanh", _gelu_no_cubic),
+    "gelu_tanh: sign of tanh flipped": ("gelu_tanh", _gelu_sign),
+    "mlp_delta: delta sign flipped": ("mlp_delta", _mlp_delta_sign),
+    "mlp_delta: bias b1 dropped": ("mlp_delta", _mlp_delta_no_bias),
+    "mlp_delta: cache not written back": ("mlp_delta", _mlp_delta_stale_cache),
+    "topk_cols: ties to the higher index": ("topk_cols", _topk_high_ties),
+    "topk_cols: indices not ascending": ("topk_cols", _topk_unsorted),
+    "ordered_key: -0 not equal to +0": ("ordered_key", _key_no_neg_zero),
+    "merge_partials: weights inverted": ("merge_partials", _merge_wrong_weight),
+    "attn_partial: logit scale dropped": ("attn_partial", _partial_no_scale),
+    "attn_mass: softmax over the wrong axis": ("attn_mass", _mass_wrong_axis),
+    "complement_partial: selected keys kept": ("complement_partial", _complement_keeps_selected),
+    "mlp_scores: absolute value dropped": ("mlp_scores", _scores_no_abs),
+    "bf16_round: truncation instead of nearest-even": ("bf16_round", _bf16_truncate),
+}
+
+
+@pytest.mark.parametrize("what", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(monkeypatch, what):
+    fname, mutant = MUTATIONS[what]
+    failed = _caught(monkeypatch, fname, mutant)
+    assert failed, f"no pin caught: {what}"
+
+
+def test_unmutated_oracle_passes_every_pin(monkeypatch):
+    assert _caught(monkeypatch, "gelu_tanh", OC.gelu_tanh) == []

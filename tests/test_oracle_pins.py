@@ -362,3 +362,16 @@ def test_attn_refresh_complement_and_selection():
             keys = [j for j in range(24) if j not in sel]
             brute = _softmax_attention_brute(q[hh, list(rows)], k[hh], v[hh], 0.5, keys=keys)
             np.testing.assert_allclose(r["acc_c"][hh, 8 * b:8 * b + 8] / r["l_c"][hh, 8 * b:8 * b + 8, None], brute, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- input generator
+
+def test_generator_draws_at_counters_match_the_stream():
+    from dynamic_column_sparse_b200 import synth
+    full = synth.normal_bf16(9, 5, (40, 24), std=0.5)
+    rows = np.array([0, 7, 39])
+    np.testing.assert_array_equal(synth.rows_bf16(9, 5, 24, rows, std=0.5), full[rows])
+    drifted = synth.drift_bf16(full, 10, 6, 0.03)
+    np.testing.assert_array_equal(synth.drift_rows_bf16(full[rows], 10, 6, 24, rows, 0.03), drifted[rows])
+    z = synth.normal_f64(3, 4, 1 << 21)
+    assert abs(z.mean()) < 3e-3 and abs(z.std() - 1.0) < 3e-3
