@@ -530,6 +530,32 @@ def extra_rows(L, w, peaks, flush, torch, cm):
     rows["dense_layer_k_all"] = {"us": round((ms_dm + ms_da) * 1e3, 1), "mlp_us": round(ms_dm * 1e3, 1),
                                  "attn_us": round(ms_da * 1e3, 1),
                                  "tflops": round((dense_mlp_f + dense_attn_f) / ((ms_dm + ms_da) * 1e-3) / 1e12, 1)}
+    # multi-step schedule (10 steps, dense at 0 and 5) across sparsity levels, through the layer API
+    from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaAttention, SparseDeltaMLP
+    sweep = {}
+    dense_us = (ms_dm + ms_da) * 1e3
+    for mp, ap in ((500, 500), (300, 165), (150, 150), (70, 70)):
+        mlp = SparseDeltaMLP(L.w1t, L.b1, L.w2, L.b2, T, Bt, mp)
+        att = SparseDeltaAttention(T, h, L.dev, ap)
+        mlp.refresh(L.x_prev)
+        att.refresh(*L.qkv_prev)
+        ms_ref = time_events(lambda: (mlp.refresh(L.x_prev), att.refresh(*L.qkv_prev)), 3, flush, torch)
+        it = [0]
+
+        def sparse_step():
+            i = it[0] = it[0] + 1
+            mlp.step(L.xs[i % 2])
+            att.step(*L.qkvs[i % 2])
+        ms_sp = time_events(sparse_step, reps, flush, torch)
+        sched = Schedule((0, 5))
+        n_dense = sum(sched.is_dense(s) for s in range(10))
+        amort = (n_dense * ms_ref + (10 - n_dense) * ms_sp) / 10 * 1e3
+        sweep[f"mlp{100 - mp // 10}_attn{round(100 - ap / 10, 1)}"] = {
+            "mlp_k": mlp.k, "attn_k": att.k, "sparse_step_us": round(ms_sp * 1e3, 1),
+            "refresh_us": round(ms_ref * 1e3, 1), "loop10_us_per_layer_step": round(amort, 1),
+            "speedup_vs_dense_k_all": round(dense_us / (ms_sp * 1e3), 2)}
+        del mlp, att
+    rows["loop_sweep"] = sweep
     xw = L.xs[0]
     w1 = L.w1t.t()
     ms_cub = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),

@@ -2,11 +2,14 @@
 inputs drifting each step (x_{s+1} = x_s + 0.03 N(0,1)).
 
 The GPU chain (SparseDeltaMLP / SparseDeltaAttention over the C ABI) and the
-oracle chain (fp64 caches, its own selections) run the same schedule from the
-same inputs; every step's outputs must agree within the parity bar. The
-chains select independently, so a near-tie may pick a different column on
-each side; the bar absorbs that. The gap to a fully dense fp64 run (the
-method's own approximation error) is printed for information.
+oracle chain (fp64 arithmetic, its own selections) run the same schedule from
+the same inputs; every step's outputs must agree within the parity bar.
+Between steps the oracle chain keeps its caches at the library's storage
+precision (activation cache bf16, output cache and attention partial fp32),
+so that the refresh's selection, a decision taken on float scores, is taken
+on the same cache values on both sides; a remaining near-tie may still pick a
+different column and the bar absorbs that. The gap to a fully dense fp64 run
+(the method's own approximation error) is printed for information.
 """
 import math
 
@@ -54,6 +57,8 @@ def run_mlp_loop(T, D, H, permille, seed=3):
         else:
             A, Y = O.mlp_delta(x, W1, B1, W2, idx, A, Y, 128)
         ratio, _ = assert_parity(out, Y, f"MLP output, step {s}", bf16_out=True)
+        A = O.bf16_decode(O.bf16_round(A))           # caches at storage precision between steps
+        Y = O.f32(Y).astype(np.float64)
         _, dense = O.dense_mlp(x, W1, B1, W2, B2)
         gap = float(np.sqrt(np.mean((Y - dense) ** 2) / np.mean(dense ** 2)))
         worst = max(worst, ratio)
@@ -77,7 +82,8 @@ def run_attn_loop(T, h, permille, seed=4):
         q, k, v = (np.ascontiguousarray(O.bf16_decode(chains[n][s]).transpose(1, 0, 2)) for n in ("q", "k", "v"))
         if sched.is_dense(s):
             r = O.attn_refresh(q, k, v, scale, 128, kk)
-            cache, ref = (r["idx"], r["m_c"], r["l_c"], r["acc_c"]), r["O"]
+            f = lambda a: O.f32(a).astype(np.float64)  # the partial is stored as fp32
+            cache, ref = (r["idx"], f(r["m_c"]), f(r["l_c"]), f(r["acc_c"])), r["O"]
         else:
             ref = O.attn_delta(q, k, v, *cache, scale, 128)
         ratio, _ = assert_parity(out, ref, f"attention output, step {s}", bf16_out=True)
