@@ -31,7 +31,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two 64-column swizzle halves)
 constexpr float kRescaleLog2 = 8.0f;     // O and l are rescaled only when the row max grows by more than 2^8
 
-// Shared memory: Q | K[2] | V[2] | P | barriers | key-index ring [2][128] |
+// Shared memory: Q | K[2] | V[2] | P | barriers | key-index ring [4][128] |
 // row-max exchange [2][2][128] | row-sum exchange [2][2][128] | key mask (complement pass).
 struct AttnCfg {
   static constexpr uint32_t kQOff = 0;
@@ -40,7 +40,7 @@ struct AttnCfg {
   static constexpr uint32_t kPOff = kVOff + 2 * kTileBytes;
   static constexpr uint32_t kBarOff = kPOff + kTileBytes;
   static constexpr uint32_t kIdxOff = kBarOff + 256;
-  static constexpr uint32_t kXmaxOff = kIdxOff + 2 * 128 * 4;
+  static constexpr uint32_t kXmaxOff = kIdxOff + 4 * 128 * 4;
   static constexpr uint32_t kXsumOff = kXmaxOff + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMaskOff = kXsumOff + 2 * 2 * 128 * 4;
 };
@@ -74,19 +74,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *q_empty = bars + 1;
   uint64_t *k_full = bars + 2;     // [2]
   uint64_t *v_full = bars + 4;     // [2]
-  uint64_t *kv_empty = bars + 6;   // [2]
-  uint64_t *s_full = bars + 8;     // [2]
-  uint64_t *s_empty = bars + 10;   // [2]
-  uint64_t *o_full = bars + 12;    // [2]
-  uint64_t *o_empty = bars + 14;   // [2]
-  uint64_t *p_full = bars + 16;
-  uint64_t *p_empty = bars + 17;
-  uint64_t *pair_bar = bars + 18;  // [4]: the two softmax warps of a lane quadrant exchange row partials
-  uint64_t *kidx_bar = bars + 22;  // producers: a chunk's keys are staged
-  uint64_t *mask_bar = bars + 23;  // softmax warps: complement mask steps
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
+  uint64_t *k_empty = bars + 6;    // [2] released when S = Q K^T of the stage has been computed
+  uint64_t *v_empty = bars + 8;    // [2] released when P V of the stage has been computed
+  uint64_t *s_full = bars + 10;    // [2]
+  uint64_t *s_empty = bars + 12;   // [2]
+  uint64_t *o_full = bars + 14;    // [2]
+  uint64_t *o_empty = bars + 16;   // [2]
+  uint64_t *p_full = bars + 18;
+  uint64_t *p_empty = bars + 19;
+  uint64_t *pair_bar = bars + 20;  // [4]: the two softmax warps of a lane quadrant exchange row partials
+  uint64_t *kidx_bar = bars + 24;  // producers: a chunk's keys are staged
+  uint64_t *mask_bar = bars + 25;  // softmax warps: complement mask steps
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [2][128] selected keys of a chunk
+  int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [4][128] selected keys of chunk g at g & 3
   float *xmax = reinterpret_cast<float *>(smem + C::kXmaxOff);   // [2][2][128] partial row maxima
   float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
   uint32_t *mask = reinterpret_cast<uint32_t *>(smem + C::kMaskOff);
@@ -104,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], MODE == kAttnDelta ? kProducers : 1);
       mbar_init(&v_full[s], MODE == kAttnDelta ? kProducers : 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], kSoftmaxThreads);
       mbar_init(&o_full[s], 1);
@@ -134,27 +136,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ producers
+    // Loads in the order the MMA warp consumes them: per tile Q, K0, K1, V0,
+    // K2, V1, .., K(n-1), V(n-2), V(n-1). A K stage frees as soon as its
+    // S = Q K^T is done, a V stage only after its P V, so K runs one chunk
+    // ahead of V; the last V of a tile goes out before the next tile's loads.
+    // g counts chunks over this CTA's tiles.
     const int pw = warp - kProdWarp0;
     const int pt = threadIdx.x - kProdWarp0 * 32;  // 0..95
-    // selected keys of chunk i of tile `tile`, rows pt and pt + 96 (the latter for pt < 32)
-    auto load_keys = [&](int tile, int i, int &ka, int &kb2) {
+    const int my_tiles = static_cast<int>(blockIdx.x) < ntiles ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+    const int total = my_tiles * nchunks;
+    // selected keys of chunk g, rows pt and pt + 96 (the latter for pt < 32)
+    auto load_keys = [&](int g, int &ka, int &kb2) {
+      const int tile = blockIdx.x + (g / nchunks) * gridDim.x, i = g % nchunks;
       const int hh = tile % p.h, b = tile / p.h;
       const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
       ka = __ldg(irow + min(i * 128 + pt, p.k - 1));
       kb2 = pt < 32 ? __ldg(irow + min(i * 128 + pt + 96, p.k - 1)) : 0;
-      if (static_cast<unsigned>(ka) >= static_cast<unsigned>(T) || static_cast<unsigned>(kb2) >= static_cast<unsigned>(T)) {
-        atomicCAS(p.status, kDevOk, kDevBadIndex);
-        ka = static_cast<unsigned>(ka) >= static_cast<unsigned>(T) ? 0 : ka;
-        kb2 = static_cast<unsigned>(kb2) >= static_cast<unsigned>(T) ? 0 : kb2;
+    };
+    // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
+    auto gather = [&](const uint16_t *src, uint8_t *dst, const int *ks, int hh) {
+      const int c16 = lane & 15;
+      const uint32_t off_half = (c16 >> 3) * 16384;
+      const uint32_t d0 = smem_u32(dst);
+      for (int qp = pw; qp < 64; qp += 3) {
+        const int r = 2 * qp + (lane >> 4);
+        const size_t gsrc = (static_cast<size_t>(ks[r]) * p.h + hh) * 128 + c16 * 8;
+        cp_async_16(d0 + off_half + sw128_offset(r, c16 & 7), src + gsrc);
       }
     };
     int ka = 0, kb2 = 0;
-    if (MODE == kAttnDelta && nchunks > 0 && static_cast<int>(blockIdx.x) < ntiles) load_keys(blockIdx.x, 0, ka, kb2);
+    if (MODE == kAttnDelta && total > 0) load_keys(0, ka, kb2);
     uint32_t kidx_phase = 0;
-    int tl = 0;
+    // K of chunk g (i = its index in the tile), for the tile's head / block
+    auto load_k = [&](int g, int i, int hh) -> bool {
+      const int s = g & 1;
+      if (!wait_warp(&k_empty[s], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) return false;
+      if (MODE == kAttnDelta) {
+        // stage the chunk's keys in slot g & 3 (read again for V two loads
+        // later), range-checked, then fetch the next chunk's while the copies go out
+        if (static_cast<unsigned>(ka) >= static_cast<unsigned>(T) || static_cast<unsigned>(kb2) >= static_cast<unsigned>(T)) {
+          atomicCAS(p.status, kDevOk, kDevBadIndex);
+          ka = static_cast<unsigned>(ka) >= static_cast<unsigned>(T) ? 0 : ka;
+          kb2 = static_cast<unsigned>(kb2) >= static_cast<unsigned>(T) ? 0 : kb2;
+        }
+        int *ks = kidx + (g & 3) * 128;
+        ks[pt] = ka;
+        if (pt < 32) ks[pt + 96] = kb2;
+        mbar_arrive(kidx_bar);
+        if (!wait_warp(kidx_bar, kidx_phase & 1, p.status, abort_flag)) return false;
+        ++kidx_phase;
+        if (g + 1 < total) load_keys(g + 1, ka, kb2);
+        gather(p.k_ptr, sK + s * kTileBytes, ks, hh);
+        cp_async_arrive_noinc(&k_full[s]);
+      } else if (pw == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
+        tma_load_2d(sK + s * kTileBytes, &tm_k, &k_full[s], hh * 128, i * 128);
+        tma_load_2d(sK + s * kTileBytes + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto load_v = [&](int g, int i, int hh) -> bool {
+      const int s = g & 1;
+      if (!wait_warp(&v_empty[s], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) return false;
+      if (MODE == kAttnDelta) {
+        gather(p.v_ptr, sV + s * kTileBytes, kidx + (g & 3) * 128, hh);
+        cp_async_arrive_noinc(&v_full[s]);
+      } else if (pw == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&v_full[s], kTileBytes);
+        tma_load_2d(sV + s * kTileBytes, &tm_v, &v_full[s], hh * 128, i * 128);
+        tma_load_2d(sV + s * kTileBytes + 16384, &tm_v, &v_full[s], hh * 128 + 64, i * 128);
+      }
+      __syncwarp();
+      return true;
+    };
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
-      if (nchunks == 0) continue;
+    int g0 = 0;
+    for (int tl = 0; tl < my_tiles && ok && nchunks > 0; ++tl, g0 += nchunks) {
+      const int tile = blockIdx.x + tl * gridDim.x;
       const int hh = tile % p.h, b = tile / p.h;
       if (pw == 0) {
         if (!wait_warp(q_empty, (tl & 1) ^ 1, p.status, abort_flag)) break;
@@ -165,56 +224,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      for (int i = 0; i < nchunks; ++i) {
-        const int g = tl * nchunks + i, s = g & 1;
-        if (!wait_warp(&kv_empty[s], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) {
+      if (MODE == kAttnDelta && pw == 1 && lane == 0) {
+        // the merge epilogue of this tile reads its rows of the complement accumulator
+        const int nrows = min(128, T - b * 128);
+        prefetch_l2_bulk(p.acc_c + (static_cast<size_t>(hh) * T + b * 128) * 128, static_cast<uint32_t>(nrows) * 512u);
+      }
+      for (int i = 0; i <= nchunks; ++i) {
+        if (i < nchunks && !load_k(g0 + i, i, hh)) {
           ok = false;
           break;
         }
-        uint8_t *dk = sK + s * kTileBytes;
-        uint8_t *dv = sV + s * kTileBytes;
-        if (MODE == kAttnDelta) {
-          // stage this chunk's keys, then fetch the next chunk's while the copies go out
-          int *ks = kidx + s * 128;
-          ks[pt] = ka;
-          if (pt < 32) ks[pt + 96] = kb2;
-          mbar_arrive(kidx_bar);
-          if (!wait_warp(kidx_bar, kidx_phase & 1, p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          ++kidx_phase;
-          {
-            int nt = tile, ni = i + 1;
-            if (ni == nchunks) {
-              ni = 0;
-              nt = tile + gridDim.x;
-            }
-            if (nt < ntiles) load_keys(nt, ni, ka, kb2);
-          }
-          // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
-          const int c16 = lane & 15;
-          const uint32_t off_half = (c16 >> 3) * 16384;
-          const uint32_t k0 = smem_u32(dk), v0 = smem_u32(dv);
-          for (int qp = pw; qp < 64; qp += 3) {
-            const int r = 2 * qp + (lane >> 4);
-            const int key = ks[r];
-            const size_t gsrc = (static_cast<size_t>(key) * p.h + hh) * 128 + c16 * 8;
-            const uint32_t o = off_half + sw128_offset(r, c16 & 7);
-            cp_async_16(k0 + o, p.k_ptr + gsrc);
-            cp_async_16(v0 + o, p.v_ptr + gsrc);
-          }
-          cp_async_arrive_noinc(&k_full[s]);
-          cp_async_arrive_noinc(&v_full[s]);
-        } else if (pw == 0 && lane == 0) {
-          mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-          tma_load_2d(dk, &tm_k, &k_full[s], hh * 128, i * 128);
-          tma_load_2d(dk + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
-          mbar_arrive_expect_tx(&v_full[s], kTileBytes);
-          tma_load_2d(dv, &tm_v, &v_full[s], hh * 128, i * 128);
-          tma_load_2d(dv + 16384, &tm_v, &v_full[s], hh * 128 + 64, i * 128);
+        if (i >= 1 && !load_v(g0 + i - 1, i - 1, hh)) {
+          ok = false;
+          break;
         }
-        __syncwarp();
       }
     }
   } else if (warp == kMmaWarp) {
@@ -246,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         kk > 0);
             }
             umma_commit(&s_full[s]);
+            umma_commit(&k_empty[s]);
             if (i == nchunks - 1) umma_commit(q_empty);
           }
           __syncwarp();
@@ -265,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 0; kk < 8; ++kk)
               umma_bf16(tO, sdesc_sw128(p0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                         sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV, (j | kk) != 0);
-            umma_commit(&kv_empty[s]);
+            umma_commit(&v_empty[s]);
             umma_commit(p_empty);
             if (j == nchunks - 1) umma_commit(&o_full[ob]);
           }
@@ -317,6 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicCAS(p.status, kDevOk, kDevBadIndex);
         }
         if (!mask_sync()) break;
+      }
+      // this row's cached complement statistics, needed only by the final merge
+      const size_t row = static_cast<size_t>(hh) * T + gi;
+      float mc = 0.f, lc = 0.f;
+      if (MODE == kAttnDelta && gi < T) {
+        mc = p.m_c[row];
+        lc = p.l_c[row];
       }
       float m_used = -INFINITY, l = 0.f;   // m_used in log2 units of the scaled logits
       for (int i = 0; i < nchunks; ++i) {
@@ -422,61 +453,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       xs[half * 128 + r] = l;
       if (!pair_sync()) break;
       l += xs[(half ^ 1) * 128 + r];
-      float ov[64];
+      // complement accumulator row, this half's 64 dimensions: the first 32 are
+      // loaded while P V of the last chunk runs, the rest (already pulled into
+      // L2 by the producers at the start of the tile) when they are merged
+      const float4 *acg = reinterpret_cast<const float4 *>(p.acc_c + row * 128 + half * 64);
+      float4 acv[8];
+      if (MODE == kAttnDelta && gi < T) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) acv[e4] = acg[e4];
+      }
       if (nchunks > 0) {
         if (!wait_warp(&o_full[ob], (tl >> 1) & 1, p.status, abort_flag)) break;
         tc_fence_after();
-        tmem_ld32_async(tO, ov);
-        tmem_ld32_async(tO + 32, ov + 32);
-        tmem_wait_ld_regs(ov);
-        reg_fence32(ov + 32);
-        tc_fence_before();
-        mbar_arrive(&o_empty[ob]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) ov[e] = 0.f;
       }
-      if (gi < T) {
-        const size_t row = static_cast<size_t>(hh) * T + gi;
-        const float m2 = m_used;
-        const int d0 = half * 64;
-        if (MODE == kAttnDelta) {
-          const float mc = p.m_c[row], lc = p.l_c[row];
-          const float mc2 = mc * kLog2e;
-          const float M = fmaxf(mc2, m2);
-          const float wc = (mc == -INFINITY) ? 0.f : exp2_approx(mc2 - M);
-          const float ws = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - M);
-          const float L = lc * wc + l * ws;
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          const float4 *ac = reinterpret_cast<const float4 *>(p.acc_c + row * 128 + d0);
-          uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
+      const float m2 = m_used;
+      float wc = 0.f, ws = 0.f, inv = 0.f;
+      if (MODE == kAttnDelta) {
+        const float mc2 = mc * kLog2e;
+        const float M = fmaxf(mc2, m2);
+        wc = (mc == -INFINITY) ? 0.f : exp2_approx(mc2 - M);
+        ws = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - M);
+        const float L = lc * wc + l * ws;
+        inv = L > 0.f ? 1.f / L : 0.f;
+      } else if (MODE == kAttnDense) {
+        inv = l > 0.f ? 1.f / l : 0.f;
+      }
+      // O of this half in two groups of 32 dimensions
 #pragma unroll
-          for (int e8 = 0; e8 < 8; ++e8) {
-            const float4 a0 = ac[2 * e8], a1 = ac[2 * e8 + 1];
-            const float *oa = ov + 8 * e8;
-            orow[e8] = make_uint4(cvt_bf16x2((a0.x * wc + oa[0] * ws) * inv, (a0.y * wc + oa[1] * ws) * inv),
-                                  cvt_bf16x2((a0.z * wc + oa[2] * ws) * inv, (a0.w * wc + oa[3] * ws) * inv),
-                                  cvt_bf16x2((a1.x * wc + oa[4] * ws) * inv, (a1.y * wc + oa[5] * ws) * inv),
-                                  cvt_bf16x2((a1.z * wc + oa[6] * ws) * inv, (a1.w * wc + oa[7] * ws) * inv));
+      for (int c = 0; c < 2; ++c) {
+        float ov[32];
+        if (nchunks > 0) {
+          tmem_ld32(tO + c * 32, ov);
+          if (c == 1) {
+            tc_fence_before();
+            mbar_arrive(&o_empty[ob]);
           }
-        } else if (MODE == kAttnDense) {
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-          uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
-#pragma unroll
-          for (int e8 = 0; e8 < 8; ++e8) {
-            const float *oa = ov + 8 * e8;
-            orow[e8] = make_uint4(cvt_bf16x2(oa[0] * inv, oa[1] * inv), cvt_bf16x2(oa[2] * inv, oa[3] * inv),
-                                  cvt_bf16x2(oa[4] * inv, oa[5] * inv), cvt_bf16x2(oa[6] * inv, oa[7] * inv));
-          }
-          if (half == 0) p.lse[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
         } else {
-          if (half == 0) {
-            p.m_c[row] = (m2 == -INFINITY) ? -INFINITY : m2 * kLn2;
-            p.l_c[row] = l;
-          }
-          float4 *ac = reinterpret_cast<float4 *>(p.acc_c + row * 128 + d0);
 #pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) ac[e4] = make_float4(ov[4 * e4], ov[4 * e4 + 1], ov[4 * e4 + 2], ov[4 * e4 + 3]);
+          for (int e = 0; e < 32; ++e) ov[e] = 0.f;
+        }
+        if (gi < T) {
+          const int d0 = half * 64 + c * 32;
+          if (MODE == kAttnDelta) {
+            uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) {
+              const float4 a0 = c == 0 ? acv[2 * e8] : acg[8 + 2 * e8];
+              const float4 a1 = c == 0 ? acv[2 * e8 + 1] : acg[9 + 2 * e8];
+              const float *oa = ov + 8 * e8;
+              orow[e8] = make_uint4(cvt_bf16x2((a0.x * wc + oa[0] * ws) * inv, (a0.y * wc + oa[1] * ws) * inv),
+                                    cvt_bf16x2((a0.z * wc + oa[2] * ws) * inv, (a0.w * wc + oa[3] * ws) * inv),
+                                    cvt_bf16x2((a1.x * wc + oa[4] * ws) * inv, (a1.y * wc + oa[5] * ws) * inv),
+                                    cvt_bf16x2((a1.z * wc + oa[6] * ws) * inv, (a1.w * wc + oa[7] * ws) * inv));
+            }
+          } else if (MODE == kAttnDense) {
+            uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) {
+              const float *oa = ov + 8 * e8;
+              orow[e8] = make_uint4(cvt_bf16x2(oa[0] * inv, oa[1] * inv), cvt_bf16x2(oa[2] * inv, oa[3] * inv),
+                                    cvt_bf16x2(oa[4] * inv, oa[5] * inv), cvt_bf16x2(oa[6] * inv, oa[7] * inv));
+            }
+          } else {
+            float4 *ac = reinterpret_cast<float4 *>(p.acc_c + row * 128 + d0);
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4)
+              ac[e4] = make_float4(ov[4 * e4], ov[4 * e4 + 1], ov[4 * e4 + 2], ov[4 * e4 + 3]);
+          }
+        }
+      }
+      if (gi < T && half == 0) {
+        if (MODE == kAttnDense) {
+          p.lse[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
+        } else if (MODE == kAttnComplement) {
+          p.m_c[row] = (m2 == -INFINITY) ? -INFINITY : m2 * kLn2;
+          p.l_c[row] = l;
         }
       }
     }

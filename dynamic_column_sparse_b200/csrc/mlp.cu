@@ -1,15 +1,15 @@
 // mlp.cu - gathered-column MLP kernels of the sparse delta step and the refresh.
 //
-// Kernel 1 (mlp_up): one CTA per (token block b, chunk of 128 selected hidden
-// columns). The 128 selected rows of W1^T are gathered into a 128-byte-
-// swizzled shared tile by four producer warps with 16-byte cp.async (each
-// warp instruction moves four whole 128-byte row segments); on a refresh,
-// where the rows are consecutive, one TMA tile load brings them instead. The
-// token block of x arrives by a tiled TMA load. One thread issues tcgen05 bf16
-// MMAs accumulating D[col][token] in TMEM. The epilogue warps own one hidden
-// column each (one TMEM lane) and all Bt tokens of it, so the activation cache
-// run a_cache[b][c][0..Bt) and the delta row are read and written as whole
-// contiguous runs.
+// Kernel 1 (mlp_up): tiles (token block b, chunk of 128 selected hidden
+// columns), walked by persistent CTAs. The 128 selected rows of W1^T are
+// gathered into a 128-byte-swizzled shared tile by four producer warps with
+// 16-byte cp.async (each warp instruction moves four whole 128-byte row
+// segments); on a refresh, where the rows are consecutive, one TMA tile load
+// brings them instead. The token block of x arrives by a tiled TMA load. One
+// thread issues tcgen05 bf16 MMAs accumulating D[col][token] in one of two
+// TMEM accumulators. Each epilogue thread owns one hidden column (one TMEM
+// lane) and half of the block's tokens, so the activation cache run
+// a_cache[b][c][..] and the delta row are read and written as contiguous runs.
 //
 // Kernel 2 (mlp_down): one CTA per (token block b, slice of BN model columns).
 // K runs over the selected hidden units: the delta rows come from the
@@ -19,11 +19,9 @@
 // cache (or overwrites it with result + b2 on a refresh) and writes the bf16
 // layer output.
 //
-// Each kernel keeps two shared-memory rings: a deep one for the gathered
-// operand (filled by producer warps 0-3 with cp.async) and a shallow one for
-// the operand that arrives by tiled TMA (issued by warp 9), so that more
-// gathered bytes are in flight. Warp 4 = MMA issuer and TMEM owner, warps
-// 5-8 = epilogue (TMEM lane quadrant = warp % 4).
+// Each kernel keeps two shared-memory rings: one for the gathered operand
+// (filled by the cp.async producer warps) and one for the operand that
+// arrives by tiled TMA. The warp roles are listed with `Roles` below.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -32,10 +30,21 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kProducers = 128;
-constexpr int kMmaWarp = 4;
-constexpr int kTmaWarp = 9;
+// Warp roles of both kernels: warps 0 .. P-1 gather with cp.async, warp P
+// issues the MMAs and owns TMEM, warps P+1 .. P+E run the epilogue (TMEM lane
+// quadrant = warp % 4; with E = 8 two warps share a quadrant, one per half of
+// the accumulator columns), warp P+E+1 issues the TMA loads.
+template <int P, int E>
+struct Roles {
+  static constexpr int kProdWarps = P;
+  static constexpr int kProducers = 32 * P;
+  static constexpr int kMmaWarp = P;
+  static constexpr int kEpiWarp0 = P + 1;
+  static constexpr int kEpiWarps = E;
+  static constexpr int kTmaWarp = P + 1 + E;
+  static constexpr int kThreads = 32 * (P + 2 + E);
+};
+
 constexpr int kBK = 64;  // K elements per pipeline stage = one 128-byte swizzle row
 
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
@@ -45,45 +54,59 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *s
 }
 
 template <int BT>
-struct UpCfg {
-  static constexpr int kStagesA = BT == 128 ? 4 : 5;  // gathered W1^T rows
-  static constexpr int kStagesB = 2;                  // x tile
+struct UpCfg : Roles<4, 4> {
+  static constexpr int kCtasPerSm = 2;                // two independent pipelines per SM
+  static constexpr int kStagesA = BT == 128 ? 3 : 4;  // gathered W1^T rows
+  static constexpr int kStagesB = BT == 128 ? 3 : 4;  // x tile
   static constexpr uint32_t kABytes = 128 * 128;      // 128 gathered rows x 64 bf16
   static constexpr uint32_t kBBytes = BT * 128;       // BT tokens x 64 bf16
   static constexpr uint32_t kBOff = kStagesA * kABytes;
-  static constexpr uint32_t kBarOff = kBOff + kStagesB * kBBytes;
+  static constexpr uint32_t kPartOff = kBOff + kStagesB * kBBytes;  // [2][128] fp32 partial column scores
+  static constexpr uint32_t kBarOff = kPartOff + 2 * 128 * 4;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
 };
 
-// two CTAs per SM (registers capped at 65536 / (2 * kThreads)): one CTA's
-// epilogue overlaps the other's main loop
+// Persistent: CTA c handles tiles c, c + gridDim.x, ... where tile = chunk * nb
+// + b (chunk-major: index lists are ascending, so CTAs running at the same
+// time gather W1^T rows from the same region, for L2 reuse). Two TMEM
+// accumulators alternate between tiles, so the epilogue of one tile overlaps
+// the main loop of the next; ring stages and parities follow one running
+// k-step counter across tiles.
 template <int BT, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
     mlp_up_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
                   const MlpUpParams p) {
   using C = UpCfg<BT>;
   constexpr int SA = C::kStagesA, SB = C::kStagesB;
+  constexpr int kProducers = C::kProducers, kMmaWarp = C::kMmaWarp, kTmaWarp = C::kTmaWarp;
+  constexpr int kEpiThreads = 32 * C::kEpiWarps;
+  constexpr int kParts = C::kEpiWarps / 4;  // epilogue warps per TMEM lane quadrant
+  constexpr int kHalf = BT / kParts;         // accumulator columns (tokens) of one epilogue warp
+  constexpr int kRowIters = 1024 / kProducers;  // gathered rows of a stage per producer thread
   constexpr uint32_t kIdesc = idesc_bf16(128, BT, false, false);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
   uint8_t *sB = smem + C::kBOff;
+  float *part = reinterpret_cast<float *>(smem + C::kPartOff);
   uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
   uint64_t *a_empty = a_full + SA;
   uint64_t *b_full = a_empty + SA;
   uint64_t *b_empty = b_full + SB;
-  uint64_t *acc_full = b_empty + SB;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  uint64_t *acc_full = b_empty + SB;   // [2]
+  uint64_t *acc_empty = acc_full + 2;  // [2]
+  uint64_t *part_bar = acc_empty + 2;  // refresh: both token halves of every column have their partial score
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(part_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *rows = reinterpret_cast<int *>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  // chunk-major across blocks: index lists are ascending, so CTAs running at
-  // the same time gather W1^T rows from the same region (L2 reuse)
-  const int chunk = blockIdx.x / p.nb;
-  const int b = blockIdx.x % p.nb;
   const bool sparse = p.mode == kUpDelta;
+  const int ntiles = p.nb * p.nchunks;
+  const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
+                           ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                           : 0;
+  const int nk = p.D / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -94,7 +117,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], kEpiThreads);
+    }
+    mbar_init(part_bar, kEpiThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -103,130 +130,189 @@ __global__ void __launch_bounds__(kThreads, 2)
     prefetch_tmap(&tm_x);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, BT);
+    tmem_alloc(tmem_slot, 2 * BT);
     tmem_relinquish();
-  }
-  if (threadIdx.x < 128) {
-    const int j = chunk * 128 + threadIdx.x;
-    int c;
-    if (sparse) {
-      c = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
-      if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights / cache
-        atomicCAS(p.status, kDevOk, kDevBadIndex);
-        c = 0;
-      }
-    } else {
-      c = min(j, p.H - 1);
-    }
-    rows[threadIdx.x] = c;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nk = p.D / kBK;
 
-  if (warp < 4) {
-    // gathered W1^T rows: thread pt moves 16-byte chunk (pt & 7) of rows i*16 + (pt >> 3), i = 0..7
+  if (warp < C::kProdWarps) {
+    // gathered W1^T rows: thread pt moves 16-byte chunk (pt & 7) of rows
+    // i * (kProducers / 8) + (pt >> 3), i = 0 .. kRowIters - 1
     if (!DENSE) {
       const int pt = threadIdx.x;
-      const uint16_t *src_row[8];
-      uint32_t dst_off[8];
+      uint32_t dst_off[kRowIters];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = i * 16 + (pt >> 3);
-        src_row[i] = p.w1t + static_cast<size_t>(rows[r]) * p.D + (pt & 7) * 8;
-        dst_off[i] = sw128_offset(r, pt & 7);
-      }
+      for (int i = 0; i < kRowIters; ++i) dst_off[i] = sw128_offset(i * (kProducers / 8) + (pt >> 3), pt & 7);
+      // this thread's selected columns of the CTA's tile tl, loaded one tile
+      // ahead and range-checked when they are used
+      auto load_rows = [&](int tl, int *c) {
+        const int tile = blockIdx.x + tl * gridDim.x;
+        const int chunk = tile / p.nb, b = tile % p.nb;
+#pragma unroll
+        for (int i = 0; i < kRowIters; ++i)
+          c[i] = tl < my_tiles ? __ldg(p.idx + static_cast<size_t>(b) * p.k +
+                                      min(chunk * 128 + i * (kProducers / 8) + (pt >> 3), p.k - 1))
+                               : 0;
+      };
+      int nxt[kRowIters];
+      load_rows(0, nxt);
       const uint32_t a_base = smem_u32(sA);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % SA;
-        if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
-        const uint32_t stage = a_base + s * C::kABytes;
+      int kg = 0;
+      bool ok = true;
+      for (int tl = 0; tl < my_tiles && ok; ++tl) {
+        const uint16_t *src_row[kRowIters];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
-        cp_async_arrive_noinc(&a_full[s]);
+        for (int i = 0; i < kRowIters; ++i) {
+          int c = nxt[i];
+          if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights
+            atomicCAS(p.status, kDevOk, kDevBadIndex);
+            c = 0;
+          }
+          src_row[i] = p.w1t + static_cast<size_t>(c) * p.D + (pt & 7) * 8;
+        }
+        load_rows(tl + 1, nxt);
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % SA;
+          if (!wait_warp(&a_empty[s], ((kg / SA) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t stage = a_base + s * C::kABytes;
+#pragma unroll
+          for (int i = 0; i < kRowIters; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
+          cp_async_arrive_noinc(&a_full[s]);
+        }
       }
     }
   } else if (warp == kTmaWarp) {
     // x tiles (and, on a refresh, the consecutive W1^T rows) by TMA
-    for (int kb = 0; kb < nk; ++kb) {
-      if (DENSE) {
-        const int s = kb % SA;
-        if (!wait_warp(&a_empty[s], ((kb / SA) & 1) ^ 1, p.status, abort_flag)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&a_full[s], C::kABytes);
-          tma_load_2d(sA + s * C::kABytes, &tm_w1t, &a_full[s], kb * kBK, chunk * 128);
+    int kg = 0;
+    bool ok = true;
+    for (int tl = 0; tl < my_tiles && ok; ++tl) {
+      const int tile = blockIdx.x + tl * gridDim.x;
+      const int chunk = tile / p.nb, b = tile % p.nb;
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        if (DENSE) {
+          const int s = kg % SA;
+          if (!wait_warp(&a_empty[s], ((kg / SA) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&a_full[s], C::kABytes);
+            tma_load_2d(sA + s * C::kABytes, &tm_w1t, &a_full[s], kb * kBK, chunk * 128);
+          }
         }
+        const int s = kg % SB;
+        if (!wait_warp(&b_empty[s], ((kg / SB) & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
+          tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kBK, b * BT);
+        }
+        __syncwarp();
       }
-      const int s = kb % SB;
-      if (!wait_warp(&b_empty[s], ((kb / SB) & 1) ^ 1, p.status, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
-        tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kBK, b * BT);
-      }
-      __syncwarp();
     }
   } else if (warp == kMmaWarp) {
+    int kg = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int sa = kb % SA, sb = kb % SB;
-      if (!wait_warp(&a_full[sa], (kb / SA) & 1, p.status, abort_flag) ||
-          !wait_warp(&b_full[sb], (kb / SB) & 1, p.status, abort_flag)) {
-        ok = false;
-        break;
-      }
-      if (!DENSE) fence_async_smem();
+    for (int tl = 0; tl < my_tiles && ok; ++tl) {
+      const int ab = tl & 1;
+      const uint32_t tacc = tmem + ab * BT;
+      if (!wait_warp(&acc_empty[ab], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
-        const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
-          umma_bf16(tmem, ad, bd, kIdesc, (kb | kk) != 0);
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int sa = kg % SA, sb = kg % SB;
+        if (!wait_warp(&a_full[sa], (kg / SA) & 1, p.status, abort_flag) ||
+            !wait_warp(&b_full[sb], (kg / SB) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
         }
-        umma_commit(&a_empty[sa]);
-        umma_commit(&b_empty[sb]);
+        if (!DENSE) fence_async_smem();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+          }
+          umma_commit(&a_empty[sa]);
+          umma_commit(&b_empty[sb]);
+        }
+        __syncwarp();
       }
+      if (ok && lane == 0) umma_commit(&acc_full[ab]);
       __syncwarp();
     }
-    if (ok && lane == 0) umma_commit(acc_full);
-    __syncwarp();
   } else {
+    // epilogue: thread = one selected column (TMEM lane r) and 1 / kParts of the block's tokens
+    const int ew = warp - C::kEpiWarp0;
     const int q = warp & 3;
+    const int th = ew >> 2;
     const int r = q * 32 + lane;
-    if (wait_warp(acc_full, 0, p.status, abort_flag)) {
-      tc_fence_after();
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const bool first = p.mode == kUpRefreshFirst;
+    for (int tl = 0; tl < my_tiles; ++tl) {
+      const int tile = blockIdx.x + tl * gridDim.x;
+      const int chunk = tile / p.nb, b = tile % p.nb;
+      const int ab = tl & 1;
       const int j = chunk * 128 + r;
       const bool valid_j = sparse ? (j < p.k) : (j < p.H);
-      const int c = rows[r];
-      const int nvalid = min(BT, p.T - b * BT);
-      const float bias = bf16_bits_to_f32(__ldg(p.b1 + c));
-      uint16_t *arow = p.a_cache + (static_cast<size_t>(b) * p.H + c) * BT;
-      uint16_t *drow = sparse ? p.delta + (static_cast<size_t>(b) * p.k_pad + j) * BT : nullptr;
-      const bool first = p.mode == kUpRefreshFirst;
-      float score = 0.f;
-#pragma unroll 1
-      for (int tq = 0; tq < BT / 32; ++tq) {
-        float acc[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + tq * 32, acc);
-        uint4 oldv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                         make_uint4(0, 0, 0, 0)};
-        if (valid_j && !(first && !sparse)) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(arow + tq * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) oldv[v] = src[v];
+      // column, bias and the cached activations are fetched before the accumulator is ready
+      int c;
+      if (sparse) {
+        c = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
+        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights / cache
+          atomicCAS(p.status, kDevOk, kDevBadIndex);
+          c = 0;
         }
-        const uint16_t *old = reinterpret_cast<const uint16_t *>(oldv);
+      } else {
+        c = min(j, p.H - 1);
+      }
+      const float bias = bf16_bits_to_f32(__ldg(p.b1 + c));
+      const int nvalid = min(BT, p.T - b * BT);
+      uint16_t *arow = p.a_cache + (static_cast<size_t>(b) * p.H + c) * BT + th * kHalf;
+      uint16_t *drow = sparse ? p.delta + (static_cast<size_t>(b) * p.k_pad + j) * BT + th * kHalf : nullptr;
+      // the first 32 of this warp's tokens are fetched here, the rest in the loop below
+      constexpr int kPre = 1;
+      const bool need_old = valid_j && !(first && !sparse);
+      uint4 oldv[kPre * 4];
+#pragma unroll
+      for (int v = 0; v < kPre * 4; ++v)
+        oldv[v] = need_old ? reinterpret_cast<const uint4 *>(arow)[v] : make_uint4(0, 0, 0, 0);
+      if (!wait_warp(&acc_full[ab], (tl >> 1) & 1, p.status, abort_flag)) break;
+      tc_fence_after();
+      float score = 0.f;
+#pragma unroll
+      for (int tq = 0; tq < kHalf / 32; ++tq) {
+        float acc[32];
+        tmem_ld32(tmem + lane_off + ab * BT + th * kHalf + tq * 32, acc);
+        if (tq == kHalf / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
+        }
+        uint4 oldl[4];
+        if (tq >= kPre) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            oldl[v] = need_old ? reinterpret_cast<const uint4 *>(arow + tq * 32)[v] : make_uint4(0, 0, 0, 0);
+        }
+        const uint16_t *old = reinterpret_cast<const uint16_t *>(tq < kPre ? oldv + tq * 4 : oldl);
         uint32_t na[16], dl[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           uint16_t nab[2], dlb[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int t = tq * 32 + i + u;
+            const int t = th * kHalf + tq * 32 + i + u;
             const float a = gelu_tanh(acc[i + u] + bias);
             const uint16_t abf = f32_to_bf16_bits(a);
             const bool tok = t < nvalid;
@@ -253,17 +339,28 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int v = 0; v < 4; ++v) dst[v] = make_uint4(dl[4 * v], dl[4 * v + 1], dl[4 * v + 2], dl[4 * v + 3]);
         }
       }
-      if (!sparse && valid_j) p.scores[static_cast<size_t>(b) * p.H + c] = score;
+      if (!sparse && kParts == 1) {
+        if (valid_j) p.scores[static_cast<size_t>(b) * p.H + c] = score;
+      } else if (!sparse) {
+        // the two token halves of a column add up their partial scores in a fixed order
+        float *pp = part + (tl & 1) * 128;
+        if (th == 1) pp[r] = score;
+        mbar_arrive(part_bar);
+        if (!wait_warp(part_bar, tl & 1, p.status, abort_flag)) break;
+        if (th == 0 && valid_j) p.scores[static_cast<size_t>(b) * p.H + c] = score + pp[r];
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, BT);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 2 * BT);
 }
 
 template <int BN>
-struct DownCfg {
+struct DownCfg : Roles<4, 4> {
+  static constexpr int kCtasPerSm = 1;
+  static constexpr int kAccs = 2;                        // TMEM accumulators (kAccs * BN columns)
   static constexpr int kStagesA = 3;                     // delta tile
   static constexpr int kStagesB = BN == 256 ? 5 : 8;     // gathered W2 rows
   static constexpr uint32_t kABytes = 128 * 128;         // 64 K-rows x 128 tokens (two 64-token atoms)
@@ -278,11 +375,13 @@ struct DownCfg {
 // the main loop of the next. Ring stages and their parities follow one
 // running k-step counter across tiles.
 template <int BT, int BN, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm)
     mlp_down_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w2,
                     const MlpDownParams p) {
   using C = DownCfg<BN>;
   constexpr int SA = C::kStagesA, SB = C::kStagesB;
+  constexpr int kProducers = C::kProducers, kMmaWarp = C::kMmaWarp, kTmaWarp = C::kTmaWarp, kThreads = C::kThreads;
+  constexpr int kRowsPerWarp = kBK / C::kProdWarps;   // gathered W2 rows of a stage per producer warp
   constexpr uint32_t kIdesc = idesc_bf16(128, BN, true, true);
   constexpr uint32_t kATx = (BT / 64) * 8192;
   constexpr int kChunksPerRow = BN / 8;               // 16-byte chunks of one gathered W2 row segment
@@ -327,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_w2);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, C::kAccs * BN);
     tmem_relinquish();
   }
   if (BT == 64) {
@@ -345,50 +444,69 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // slice-major across blocks: CTAs running at the same time share an N slice
   // and sweep their (ascending) W2 rows in the same order (L2 reuse)
-  if (warp < 4) {
-    // gathered W2 rows: warp pw moves rows pw*16 .. pw*16+15 of each 64-row stage
+  if (warp < C::kProdWarps) {
+    // gathered W2 rows: warp pw moves rows pw*R .. pw*R+R-1 (R = kRowsPerWarp) of each 64-row stage
     if (!DENSE) {
       const int pw = warp;
       const int csub = lane % kChunksPerRow;           // chunk of the row segment this lane moves
       const int rsub = lane / kChunksPerRow;           // row within one instruction
       const uint32_t b_base = smem_u32(sB);
-      int kg = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
-        const int32_t *irow = p.idx + static_cast<size_t>(b) * p.k;
-        auto load_idx = [&](int kb) -> int {           // lane < 16: index of row pw*16 + lane of stage kb
-          int c = 0;
-          if (lane < 16 && kb < nk) {
-            c = __ldg(irow + min(kb * kBK + pw * 16 + lane, p.k - 1));
-            if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
-              atomicCAS(p.status, kDevOk, kDevBadIndex);
-              c = 0;
-            }
-          }
-          return c;
-        };
-        int c_cur = load_idx(0);
-        for (int kb = 0; kb < nk; ++kb, ++kg) {
-          const int s = kg % SB;
-          const int c_next = load_idx(kb + 1);
-          if (!wait_warp(&b_empty[s], ((kg / SB) & 1) ^ 1, p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t stage = b_base + s * C::kBBytes;
-#pragma unroll
-          for (int i = 0; i < 16 / kRowsPerInstr; ++i) {
-            const int rr = i * kRowsPerInstr + rsub;   // 0..15 within this warp's rows
-            const int r = pw * 16 + rr;                // row of the stage
-            const int c = __shfl_sync(0xffffffffu, c_cur, rr);
-            const int slab = csub >> 3, cc = csub & 7;
-            cp_async_16(stage + slab * 8192 + sw128_offset(r, cc),
-                        p.w2 + static_cast<size_t>(c) * p.D + n0 + csub * 8);
-          }
-          cp_async_arrive_noinc(&b_full[s]);
-          c_cur = c_next;
+      const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
+                               ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                               : 0;
+      const int total = my_tiles * nk;
+      // Stage kg runs over this CTA's tiles; lanes < R hold the index of row
+      // pw*R + lane. Each index is loaded four stages before its copies are
+      // issued, into a register nothing reads until then (the loop body is
+      // unrolled four times, so no move waits on a pending load); its range
+      // is checked only when it is used.
+      int ltile = blockIdx.x, lkb = 0;                 // stage whose index is loaded next
+      auto load_idx = [&]() -> int {
+        int c = 0;
+        if (lane < kRowsPerWarp && ltile < ntiles)
+          c = __ldg(p.idx + static_cast<size_t>(ltile % p.nb) * p.k + min(lkb * kBK + pw * kRowsPerWarp + lane, p.k - 1));
+        if (++lkb == nk) {
+          lkb = 0;
+          ltile += gridDim.x;
         }
+        return c;
+      };
+      int tile = blockIdx.x, kb = 0;                   // stage whose copies are issued next
+      auto issue = [&](int kg, int c) -> bool {
+        const int s = kg % SB;
+        const int n0 = (tile / p.nb) * BN;
+        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
+          atomicCAS(p.status, kDevOk, kDevBadIndex);
+          c = 0;
+        }
+        if (!wait_warp(&b_empty[s], ((kg / SB) & 1) ^ 1, p.status, abort_flag)) return false;
+        const uint32_t stage = b_base + s * C::kBBytes;
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp / kRowsPerInstr; ++i) {
+          const int rr = i * kRowsPerInstr + rsub;   // row within this warp's rows
+          const int r = pw * kRowsPerWarp + rr;      // row of the stage
+          const int cr = __shfl_sync(0xffffffffu, c, rr);
+          const int slab = csub >> 3, cc = csub & 7;
+          cp_async_16(stage + slab * 8192 + sw128_offset(r, cc),
+                      p.w2 + static_cast<size_t>(cr) * p.D + n0 + csub * 8);
+        }
+        cp_async_arrive_noinc(&b_full[s]);
+        if (++kb == nk) {
+          kb = 0;
+          tile += gridDim.x;
+        }
+        return true;
+      };
+      int c0 = load_idx(), c1 = load_idx(), c2 = load_idx(), c3 = load_idx();
+      for (int kg = 0; kg < total; kg += 4) {
+        if (!issue(kg, c0)) break;
+        c0 = load_idx();
+        if (kg + 1 >= total || !issue(kg + 1, c1)) break;
+        c1 = load_idx();
+        if (kg + 2 >= total || !issue(kg + 2, c2)) break;
+        c2 = load_idx();
+        if (kg + 3 >= total || !issue(kg + 3, c3)) break;
+        c3 = load_idx();
       }
     }
   } else if (warp == kTmaWarp) {
@@ -429,9 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kg = 0, tl = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
-      const int ab = tl & 1;
+      const int ab = tl % C::kAccs;
       const uint32_t tacc = tmem + ab * BN;
-      if (!wait_warp(&acc_empty[ab], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
+      if (!wait_warp(&acc_empty[ab], ((tl / C::kAccs) & 1) ^ 1, p.status, abort_flag)) break;
       tc_fence_after();
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         const int sa = kg % SA, sb = kg % SB;
@@ -465,10 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tl = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
       const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
-      const int ab = tl & 1;
+      const int ab = tl % C::kAccs;
       const int64_t grow = static_cast<int64_t>(b) * BT + t;
       const bool valid = t < BT && grow < p.T;
-      if (!wait_warp(&acc_full[ab], (tl >> 1) & 1, p.status, abort_flag)) break;
+      if (!wait_warp(&acc_full[ab], (tl / C::kAccs) & 1, p.status, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int nc = 0; nc < BN / 32; ++nc) {
@@ -511,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 2 * BN);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, C::kAccs * BN);
 }
 
 // out = bf16(y) when a sparse step selects nothing
@@ -533,8 +651,11 @@ cudaError_t launch_up_t(const MlpUpParams &p, const CUtensorMap &w, const CUtens
   using C = UpCfg<BT>;
   cudaError_t e = set_smem(mlp_up_kernel<BT, DENSE>, C::kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.nb) * p.nchunks;
-  mlp_up_kernel<BT, DENSE><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(w, x, p);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.nchunks, static_cast<int64_t>(sms) * C::kCtasPerSm);
+  mlp_up_kernel<BT, DENSE><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, s>>>(w, x, p);
   return cudaGetLastError();
 }
 
@@ -546,8 +667,8 @@ cudaError_t launch_down_t(const MlpDownParams &p, const CUtensorMap &a, const CU
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.n_slices, sms);
-  mlp_down_kernel<BT, BN, DENSE><<<static_cast<unsigned>(grid), kThreads, C::kSmem, s>>>(a, w, p);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.n_slices, static_cast<int64_t>(sms) * C::kCtasPerSm);
+  mlp_down_kernel<BT, BN, DENSE><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, s>>>(a, w, p);
   return cudaGetLastError();
 }
 
