@@ -50,8 +50,6 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *s
   return __all_sync(0xffffffffu, ok);
 }
 
-// exp2 of 64 values in place: one in every `kFmaEvery` on the FMA pipe, the rest on MUFU
-constexpr int kFmaEvery = 5;
 
 // Persistent: each CTA walks tiles (head, 128-query block) blockIdx.x,
 // blockIdx.x + gridDim.x, ...; every tile has the same number of key chunks,
@@ -153,15 +151,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       ka = __ldg(irow + min(i * 128 + pt, p.k - 1));
       kb2 = pt < 32 ? __ldg(irow + min(i * 128 + pt + 96, p.k - 1)) : 0;
     };
-    // warp pw moves key rows 2q and 2q+1 for q = pw, pw+3, ..: lanes 0-15 one row, 16-31 the other
+    // warp pw moves the row pairs (2q, 2q+1), q = 22 pw .. 22 pw + 21 (< 64):
+    // lanes 0-15 the even row, 16-31 the odd one, 16 bytes each. The warp's
+    // keys are read from shared memory up front, so the copies issue back to
+    // back with one address computation each.
     auto gather = [&](const uint16_t *src, uint8_t *dst, const int *ks, int hh) {
-      const int c16 = lane & 15;
-      const uint32_t off_half = (c16 >> 3) * 16384;
-      const uint32_t d0 = smem_u32(dst);
-      for (int qp = pw; qp < 64; qp += 3) {
-        const int r = 2 * qp + (lane >> 4);
-        const size_t gsrc = (static_cast<size_t>(ks[r]) * p.h + hh) * 128 + c16 * 8;
-        cp_async_16(d0 + off_half + sw128_offset(r, c16 & 7), src + gsrc);
+      constexpr int kPairs = 22;
+      const int c16 = lane & 15, hi = lane >> 4;
+      const uint16_t *lb = src + hh * 128 + c16 * 8;
+      const size_t rs = static_cast<size_t>(p.h) * 128;
+      const uint32_t d0 = smem_u32(dst) + (c16 >> 3) * 16384;
+      const int q0 = pw * kPairs;
+      int key[kPairs];
+#pragma unroll
+      for (int i = 0; i < kPairs; ++i) key[i] = q0 + i < 64 ? ks[2 * (q0 + i) + hi] : 0;
+#pragma unroll
+      for (int i = 0; i < kPairs; ++i) {
+        if (q0 + i < 64) {
+          const int r = 2 * (q0 + i) + hi;
+          cp_async_16(d0 + sw128_offset(r, c16 & 7), lb + static_cast<size_t>(key[i]) * rs);
+        }
       }
     };
     int ka = 0, kb2 = 0;
@@ -426,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const float x = fmaf(sv[e], sl2, mneg);
-          sv[e] = (e % kFmaEvery == kFmaEvery - 1) ? exp2_fma(x) : exp2_approx(x);
+          sv[e] = exp2_approx(x);
           lp[e & 3] += sv[e];
         }
         l += (lp[0] + lp[1]) + (lp[2] + lp[3]);

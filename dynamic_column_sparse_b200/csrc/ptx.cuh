@@ -304,26 +304,6 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 8 (used to share the exponentials of a
-// softmax between the MUFU and FMA pipes). Method: Cody-Waite style range
-// reduction x = j + f with j = round(x) by the 1.5 * 2^23 shifter (f in
-// [-1/2, 1/2]); 2^f by a degree-4 polynomial fitted for this library as a
-// near-minimax approximation of relative error on [-1/2, 1/2] (max relative
-// error 2.7e-6 in fp32); 2^j added into the exponent field. x < -125 gives 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float xc = fmaxf(x, -125.0f);
-  const float t = xc + 12582912.0f;
-  const float j = t - 12582912.0f;
-  const float f = xc - j;
-  float p = 9.570096619e-03f;
-  p = fmaf(p, f, 5.591785908e-02f);
-  p = fmaf(p, f, 2.402474433e-01f);
-  p = fmaf(p, f, 6.931217909e-01f);
-  p = fmaf(p, f, 9.999992847e-01f);
-  const uint32_t jb = static_cast<uint32_t>(__float_as_int(t) - 0x4B400000) << 23;
-  return x < -125.0f ? 0.0f : __uint_as_float(__float_as_uint(p) + jb);
-}
-
 // Two fp32 values to packed bf16x2 (round to nearest even) in one conversion:
 // lo in bits 0..15, hi in bits 16..31.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {

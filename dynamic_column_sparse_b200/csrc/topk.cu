@@ -2,12 +2,17 @@
 //
 // For each row: the k largest fp32 scores, ties to the lower index, written as
 // ascending column indices. Scores become order-preserving uint32 keys; a
-// three-pass radix select (11 + 11 + 10 bits, 2048-bin shared histograms)
-// finds the exact k-th key tau and how many keys equal to tau are taken;
-// a stable block-wide compaction in index order then writes the result.
-// One CTA per row (grid-stride). Rows of up to kStagedMaxN scores are staged
-// in shared memory once; longer rows are re-read from global memory (L2) by
-// each pass.
+// radix select finds the exact k-th key tau and how many keys equal to tau are
+// taken; a stable block-wide compaction in index order then writes the result.
+//
+// Rows of up to kStagedMaxN scores are staged in shared memory once and run a
+// three-pass radix select (11 + 11 + 10 bits) there. Longer rows take two
+// vectorised passes over global memory: a 12-bit histogram finds the bucket
+// holding the k-th key, then every element at or above that bucket is copied
+// (key and index, in index order) into shared memory, where the remaining
+// 20 bits are resolved and the output is compacted. A row whose candidates do
+// not fit, or that is not 16-byte aligned, falls back to the general path that
+// re-reads the row from global memory for every radix pass.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -19,6 +24,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxBins = 2048;
 constexpr int kItems = 8;             // consecutive elements per thread in the compaction
 constexpr int kStagedMaxN = 40960;    // 160 KB of keys in shared memory
+constexpr int kLongBins = 4096;       // first digit of the long-row path: the top 12 key bits
+constexpr int kLongCap = 24576;       // long-row candidates held in shared memory (192 KB)
 
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -55,6 +62,113 @@ __device__ __forceinline__ uint64_t block_excl_scan(uint64_t v, uint64_t *warp_t
   return res;
 }
 
+// Given the histogram of the digit of the keys still in play and the number kk
+// of keys still to take, finds the digit of the kk-th largest key (s_digit)
+// and how many keys lie in higher digits (s_above). Block-wide.
+__device__ __forceinline__ void select_digit(const uint32_t *hist, int nbins, int kk, uint64_t *warp_tot,
+                                             uint32_t &s_digit, uint32_t &s_above) {
+  const int tid = threadIdx.x;
+  // thread t owns bins [nbins - (t+1)*per, nbins - t*per): thread 0 the highest
+  const int per = nbins / kThreads;
+  const int hi = nbins - tid * per;
+  uint32_t local = 0;
+  for (int b = hi - 1; b >= hi - per; --b) local += hist[b];
+  uint64_t tot;
+  const uint32_t above = static_cast<uint32_t>(block_excl_scan(local, warp_tot, tot));
+  if (above < static_cast<uint32_t>(kk) && above + local >= static_cast<uint32_t>(kk)) {
+    uint32_t cum = above;
+    for (int b = hi - 1; b >= hi - per; --b) {
+      if (cum + hist[b] >= static_cast<uint32_t>(kk)) {
+        s_digit = static_cast<uint32_t>(b);
+        s_above = cum;
+        break;
+      }
+      cum += hist[b];
+    }
+  }
+  __syncthreads();
+}
+
+// One tile of the stable compaction: thread t holds the keys of elements
+// first .. first + kItems - 1 (of n). An element is kept if its key exceeds
+// tau, or equals tau and fewer than kk equal keys precede it; out(pos, e)
+// writes output position pos for the thread's item e (element first + e).
+template <typename Out>
+__device__ __forceinline__ void compact_tile(const uint32_t *keys, int first, int n, uint32_t tau, int kk, int k,
+                                             uint32_t &run_gt, uint32_t &run_eq, uint64_t *warp_tot, Out out) {
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int e = 0; e < kItems; ++e) {
+    if (first + e < n) {
+      n_gt += keys[e] > tau;
+      n_eq += keys[e] == tau;
+    }
+  }
+  uint64_t tot;
+  const uint64_t before = block_excl_scan((static_cast<uint64_t>(n_gt) << 32) | n_eq, warp_tot, tot);
+  uint32_t gt_b = run_gt + static_cast<uint32_t>(before >> 32);
+  uint32_t eq_b = run_eq + static_cast<uint32_t>(before & 0xffffffffu);
+#pragma unroll
+  for (int e = 0; e < kItems; ++e) {
+    const int i = first + e;
+    if (i >= n) break;
+    if (keys[e] > tau) {
+      const uint32_t pos = gt_b + min(eq_b, static_cast<uint32_t>(kk));
+      if (pos < static_cast<uint32_t>(k)) out(pos, e);
+      ++gt_b;
+    } else if (keys[e] == tau) {
+      if (eq_b < static_cast<uint32_t>(kk) && gt_b + eq_b < static_cast<uint32_t>(k)) out(gt_b + eq_b, e);
+      ++eq_b;
+    }
+  }
+  run_gt += static_cast<uint32_t>(tot >> 32);
+  run_eq += static_cast<uint32_t>(tot & 0xffffffffu);
+}
+
+// Exact top-k of one row by a three-pass radix select over all n keys (read
+// from `staged` shared memory or, if STAGED is false, from global memory on
+// every pass), then a stable compaction.
+template <bool STAGED>
+__device__ void row_generic(const float *src, int32_t *dst, int n, int k, const uint32_t *staged, uint32_t *hist,
+                            uint64_t *warp_tot, uint32_t &s_digit, uint32_t &s_above) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0, mask = 0;
+  int kk = k;  // keys still to take among those matching prefix
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nbins = pass == 2 ? 1024 : 2048;
+    for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t key = STAGED ? staged[i] : ordered_key(__ldg(src + i));
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
+    }
+    __syncthreads();
+    select_digit(hist, nbins, kk, warp_tot, s_digit, s_above);
+    prefix |= s_digit << shift;
+    mask |= static_cast<uint32_t>(nbins - 1) << shift;
+    kk -= static_cast<int>(s_above);
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;
+  // stable compaction: an element is kept if its key exceeds tau, or equals
+  // tau and fewer than kk equal keys precede it
+  uint32_t run_gt = 0, run_eq = 0;
+  const int tile = kThreads * kItems;
+  for (int base = 0; base < n; base += tile) {
+    const int first = base + tid * kItems;
+    uint32_t keys[kItems];
+#pragma unroll
+    for (int e = 0; e < kItems; ++e) {
+      const int i = first + e;
+      keys[e] = i < n ? (STAGED ? staged[i] : ordered_key(__ldg(src + i))) : 0u;
+    }
+    compact_tile(keys, first, n, tau, kk, k, run_gt, run_eq, warp_tot, [&](uint32_t pos, int e) { dst[pos] = first + e; });
+  }
+  __syncthreads();
+}
+
 template <bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams p) {
   extern __shared__ uint32_t staged[];
@@ -78,82 +192,201 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams p) {
       for (int i = tid; i < n; i += kThreads) staged[i] = ordered_key(__ldg(src + i));
       __syncthreads();
     }
-    uint32_t prefix = 0, mask = 0;
-    int kk = k;  // keys still to take among those matching prefix
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int nbins = pass == 2 ? 1024 : 2048;
-      for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += kThreads) {
-        const uint32_t key = STAGED ? staged[i] : ordered_key(__ldg(src + i));
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
+    row_generic<STAGED>(src, dst, n, k, staged, hist, warp_tot, s_digit, s_above);
+  }
+}
+
+// Long rows (see the file comment). Dynamic shared memory holds the candidate
+// keys and indices: kLongCap entries each, split into one region per warp.
+__global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p) {
+  extern __shared__ uint32_t cand[];  // [kLongCap] keys, then [kLongCap] indices
+  __shared__ uint32_t hist[kLongBins];
+  __shared__ uint64_t warp_tot[kWarps + 1];
+  __shared__ uint32_t s_digit, s_above;
+  __shared__ uint32_t s_pref[kWarps + 1];  // start of warp w's candidates in the concatenated order
+  __shared__ int s_overflow;
+  constexpr int kRegion = kLongCap / kWarps;
+  constexpr int kUnroll = 8;
+  uint32_t *ckey = cand;
+  int32_t *cidx = reinterpret_cast<int32_t *>(cand + kLongCap);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = static_cast<int>(p.n);
+  const int k = p.k;
+  if (*(volatile int *)p.status != kDevOk) return;
+
+  for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+    const float *src = p.scores + row * p.ld_scores;
+    int32_t *dst = p.idx + row * p.ld_idx;
+    if (k >= n) {
+      for (int i = tid; i < n; i += kThreads) dst[i] = i;
+      continue;
+    }
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) {
+      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
+      continue;
+    }
+    const float4 *src4 = reinterpret_cast<const float4 *>(src);
+    const int n4 = n >> 2;
+    // pass 1: histogram of the top 12 bits of every key
+    for (int i = tid; i < kLongBins; i += kThreads) hist[i] = 0;
+    if (tid == 0) s_overflow = 0;
+    __syncthreads();
+    for (int i0 = tid; i0 < n4; i0 += kUnroll * kThreads) {
+      float4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      __syncthreads();
-      // thread t owns bins [nbins - (t+1)*per, nbins - t*per): thread 0 the highest
-      const int per = nbins / kThreads;
-      const int hi = nbins - tid * per;
-      uint32_t local = 0;
-      for (int b = hi - 1; b >= hi - per; --b) local += hist[b];
-      uint64_t tot;
-      const uint32_t above = static_cast<uint32_t>(block_excl_scan(local, warp_tot, tot));
-      if (above < static_cast<uint32_t>(kk) && above + local >= static_cast<uint32_t>(kk)) {
-        uint32_t cum = above;
-        for (int b = hi - 1; b >= hi - per; --b) {
-          if (cum + hist[b] >= static_cast<uint32_t>(kk)) {
-            s_digit = static_cast<uint32_t>(b);
-            s_above = cum;
-            break;
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (i0 + u * kThreads < n4) {
+          atomicAdd(&hist[ordered_key(v[u].x) >> 20], 1u);
+          atomicAdd(&hist[ordered_key(v[u].y) >> 20], 1u);
+          atomicAdd(&hist[ordered_key(v[u].z) >> 20], 1u);
+          atomicAdd(&hist[ordered_key(v[u].w) >> 20], 1u);
+        }
+      }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += kThreads) atomicAdd(&hist[ordered_key(__ldg(src + i)) >> 20], 1u);
+    __syncthreads();
+    select_digit(hist, kLongBins, k, warp_tot, s_digit, s_above);
+    const uint32_t b1 = s_digit;
+    const int kk1 = k - static_cast<int>(s_above);  // keys to take from bucket b1
+    __syncthreads();
+    // pass 2: warp w takes float4 elements [w seg, (w+1) seg) (the last warp also
+    // the < 4 trailing scalars) and appends every key in bucket b1 or above,
+    // with its index, to its own region, in index order
+    {
+      const int seg = (n4 + kWarps - 1) / kWarps;
+      const int f_lo = min(warp * seg, n4), f_hi = min(f_lo + seg, n4);
+      uint32_t *wkey = ckey + warp * kRegion;
+      int32_t *widx = cidx + warp * kRegion;
+      uint32_t wcount = 0;
+      bool over = false;
+      // appends this lane's flagged keys of one step (up to 4, elements base..base+3) in lane order
+      auto append = [&](const uint32_t *key, int base, int nvalid) {
+        uint32_t flags = 0, cnt = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < nvalid && (key[c] >> 20) >= b1) {
+            flags |= 1u << c;
+            ++cnt;
           }
-          cum += hist[b];
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (wcount + tot > static_cast<uint32_t>(kRegion)) {
+          over = true;  // warp-uniform
+          return;
+        }
+        uint32_t pos = wcount + incl - cnt;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (flags & (1u << c)) {
+            wkey[pos] = key[c];
+            widx[pos] = base + c;
+            ++pos;
+          }
+        wcount += tot;
+      };
+      for (int f0 = f_lo; f0 < f_hi && !over; f0 += kUnroll * 32) {
+        float4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int f = f0 + u * 32 + lane;
+          v[u] = f < f_hi ? __ldg(src4 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          if (over || f0 + u * 32 >= f_hi) break;  // warp-uniform
+          const int f = f0 + u * 32 + lane;
+          const uint32_t key[4] = {ordered_key(v[u].x), ordered_key(v[u].y), ordered_key(v[u].z), ordered_key(v[u].w)};
+          append(key, 4 * f, f < f_hi ? 4 : 0);
+        }
+      }
+      if (warp == kWarps - 1 && !over && 4 * n4 < n) {
+        // the (at most 3) trailing scalars, all on lane 0
+        const int nt = n - 4 * n4;
+        uint32_t key[4] = {0u, 0u, 0u, 0u};
+        if (lane == 0)
+          for (int c = 0; c < nt; ++c) key[c] = ordered_key(__ldg(src + 4 * n4 + c));
+        append(key, 4 * n4, lane == 0 ? nt : 0);
+      }
+      if (lane == 0) {
+        warp_tot[warp] = wcount;
+        if (over) s_overflow = 1;
+      }
+    }
+    __syncthreads();
+    if (s_overflow) {
+      __syncthreads();
+      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
+      continue;
+    }
+    if (tid == 0) {
+      uint32_t acc = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        s_pref[w] = acc;
+        acc += static_cast<uint32_t>(warp_tot[w]);
+      }
+      s_pref[kWarps] = acc;
+    }
+    __syncthreads();
+    const int count = static_cast<int>(s_pref[kWarps]);
+    // candidate L of the concatenated (index-ordered) list
+    auto cand_at = [&](int L, uint32_t &key, int32_t &idx) {
+      int w = 0;
+#pragma unroll
+      for (int step = kWarps / 2; step >= 1; step >>= 1)
+        if (static_cast<uint32_t>(L) >= s_pref[w + step]) w += step;
+      const int j = w * kRegion + (L - static_cast<int>(s_pref[w]));
+      key = ckey[j];
+      idx = cidx[j];
+    };
+    // the remaining 20 bits (10 + 10) among the candidates of bucket b1
+    uint32_t prefix = b1 << 20, mask = 0xfff00000u;
+    int kk = kk1;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      for (int i = tid; i < 1024; i += kThreads) hist[i] = 0;
+      __syncthreads();
+      for (int w = 0; w < kWarps; ++w) {
+        const int cw = static_cast<int>(s_pref[w + 1] - s_pref[w]);
+        for (int j = tid; j < cw; j += kThreads) {
+          const uint32_t key = ckey[w * kRegion + j];
+          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
         }
       }
       __syncthreads();
+      select_digit(hist, 1024, kk, warp_tot, s_digit, s_above);
       prefix |= s_digit << shift;
-      mask |= static_cast<uint32_t>(nbins - 1) << shift;
+      mask |= 1023u << shift;
       kk -= static_cast<int>(s_above);
       __syncthreads();
     }
     const uint32_t tau = prefix;
-    // stable compaction: an element is kept if its key exceeds tau, or equals
-    // tau and fewer than kk equal keys precede it
+    // stable compaction over the candidates in index order
     uint32_t run_gt = 0, run_eq = 0;
     const int tile = kThreads * kItems;
-    for (int base = 0; base < n; base += tile) {
+    for (int base = 0; base < count; base += tile) {
       const int first = base + tid * kItems;
       uint32_t keys[kItems];
-      uint32_t n_gt = 0, n_eq = 0;
+      int32_t ids[kItems];
 #pragma unroll
       for (int e = 0; e < kItems; ++e) {
-        const int i = first + e;
-        uint32_t key = 0;
-        if (i < n) key = STAGED ? staged[i] : ordered_key(__ldg(src + i));
-        keys[e] = key;
-        if (i < n) {
-          n_gt += key > tau;
-          n_eq += key == tau;
-        }
+        keys[e] = 0u;
+        ids[e] = 0;
+        if (first + e < count) cand_at(first + e, keys[e], ids[e]);
       }
-      uint64_t tot;
-      const uint64_t before = block_excl_scan((static_cast<uint64_t>(n_gt) << 32) | n_eq, warp_tot, tot);
-      uint32_t gt_b = run_gt + static_cast<uint32_t>(before >> 32);
-      uint32_t eq_b = run_eq + static_cast<uint32_t>(before & 0xffffffffu);
-#pragma unroll
-      for (int e = 0; e < kItems; ++e) {
-        const int i = first + e;
-        if (i >= n) break;
-        if (keys[e] > tau) {
-          const uint32_t pos = gt_b + min(eq_b, static_cast<uint32_t>(kk));
-          if (pos < static_cast<uint32_t>(k)) dst[pos] = i;
-          ++gt_b;
-        } else if (keys[e] == tau) {
-          if (eq_b < static_cast<uint32_t>(kk) && gt_b + eq_b < static_cast<uint32_t>(k)) dst[gt_b + eq_b] = i;
-          ++eq_b;
-        }
-      }
-      run_gt += static_cast<uint32_t>(tot >> 32);
-      run_eq += static_cast<uint32_t>(tot & 0xffffffffu);
+      compact_tile(keys, first, count, tau, kk, k, run_gt, run_eq, warp_tot,
+                   [&](uint32_t pos, int e) { dst[pos] = ids[e]; });
     }
     __syncthreads();
   }
@@ -181,8 +414,15 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
     topk_kernel<true><<<static_cast<unsigned>(grid), kThreads, smem, s>>>(p);
   } else {
     // one CTA per SM keeps every row being scanned resident in L2 between passes
+    const int smem = 2 * kLongCap * static_cast<int>(sizeof(uint32_t));
+    static bool long_attr_set = false;
+    if (!long_attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(topk_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      long_attr_set = true;
+    }
     const int64_t grid = std::min<int64_t>(p.rows, sms);
-    topk_kernel<false><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(p);
+    topk_long_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(p);
   }
   return cudaGetLastError();
 }

@@ -114,3 +114,23 @@ def assert_parity(got, ref, what: str, max_of_rms=MAX_ERR_OF_RMS, mean_rel=MEAN_
         assert mx <= max_of_rms * rms + 1e-30, f"{what}: max|err| {mx:.3e} > {max_of_rms} * RMS {rms:.3e}"
     assert rel <= mean_rel, f"{what}: mean rel err {rel:.3e} > {mean_rel}"
     return mx / max(rms, 1e-300), rel
+
+
+def check_selection(idx, ref_scores, k, band):
+    """idx rows: strictly ascending, k distinct; every kept score >= every dropped score - band * scale."""
+    rows, n = ref_scores.shape
+    assert idx.shape == (rows, k)
+    same = 0
+    ref_idx = O.topk_cols(O.f32(ref_scores), k)
+    for r in range(rows):
+        sel = idx[r]
+        assert np.all(np.diff(sel) > 0) and sel.min() >= 0 and sel.max() < n
+        if np.array_equal(sel, ref_idx[r]):
+            same += 1
+            continue
+        mask = np.zeros(n, dtype=bool)
+        mask[sel] = True
+        scale = max(np.abs(ref_scores[r]).max(), 1e-30)
+        if k and k < n:
+            assert ref_scores[r][mask].min() >= ref_scores[r][~mask].max() - band * scale, f"row {r}"
+    return same

@@ -2,14 +2,23 @@
 inputs drifting each step (x_{s+1} = x_s + 0.03 N(0,1)).
 
 The GPU chain (SparseDeltaMLP / SparseDeltaAttention over the C ABI) and the
-oracle chain (fp64 arithmetic, its own selections) run the same schedule from
-the same inputs; every step's outputs must agree within the parity bar.
-Between steps the oracle chain keeps its caches at the library's storage
-precision (activation cache bf16, output cache and attention partial fp32),
-so that the refresh's selection, a decision taken on float scores, is taken
-on the same cache values on both sides; a remaining near-tie may still pick a
-different column and the bar absorbs that. The gap to a fully dense fp64 run
-(the method's own approximation error) is printed for information.
+oracle chain (fp64 arithmetic) run the same schedule from the same inputs;
+every step's outputs must agree within the parity bar. Between steps the
+oracle chain keeps its caches at the library's storage precision (activation
+cache bf16, output cache and attention partial fp32).
+
+A refresh's selection is a decision taken on float scores that each side
+computes on its own, so where scores nearly tie both selections are correct.
+At every refresh the test checks what is unique, that the GPU's selection is
+exactly the top-k of the GPU's own fp32 scores, and checks the scores
+themselves against the oracle's; then both chains continue from the GPU's
+selection (on the attention side the oracle rebuilds its complement cache for
+it). After a few sparse steps the two chains' bf16 activation caches can
+differ by one ulp in places, and a column score sums |a - A_cache|, a small
+difference of close values, so the score bound here is looser than on a fresh
+cache: max |err| <= 5e-2 * RMS of the scores.
+The gap to a fully dense fp64 run (the method's own approximation error) is
+printed for information.
 """
 import math
 
@@ -18,12 +27,25 @@ import pytest
 
 import oracle as O
 from dynamic_column_sparse_b200 import synth
-from helpers import assert_parity, dev_bf16, f64_of_bf16, heads_first
+from helpers import assert_parity, dev_bf16, err_stats, f64_of_bf16, heads_first
 
 pytestmark = pytest.mark.gpu
 
 DENSE_STEPS = (0, 5)
 STEPS = 10
+SCORE_MAX_OF_RMS = 5e-2
+
+
+def check_refresh_selection(gpu_idx, gpu_scores, ref_scores, k, what):
+    """The GPU's selection is the exact top-k of its own scores, which agree with the oracle's."""
+    rows = gpu_idx.shape[0]
+    np.testing.assert_array_equal(gpu_idx, O.topk_cols(gpu_scores.reshape(rows, -1), k), err_msg=what)
+    g = gpu_scores.reshape(rows, -1).astype(np.float64)
+    r = ref_scores.reshape(rows, -1)
+    mx, rms, _ = err_stats(g, r)
+    print(f"{what}: score max|err|/rms {mx / rms:.4f}, rows as the oracle's "
+          f"{int(np.sum(np.all(gpu_idx == O.topk_cols(O.f32(r), k), axis=1)))} of {rows}")
+    assert mx <= SCORE_MAX_OF_RMS * rms, f"{what}: scores"
 
 
 def drift_chain(first_bits, seed, tid, sigma, steps):
@@ -53,7 +75,9 @@ def run_mlp_loop(T, D, H, permille, seed=3):
         x = O.bf16_decode(xs[s])
         if sched.is_dense(s):
             r = O.mlp_refresh(x, W1, B1, W2, B2, A, 128, k, first_step=A is None)
-            A, Y, idx = r["a"], r["y"], r["idx"]
+            A, Y = r["a"], r["y"]
+            idx = layer.idx.cpu().numpy()
+            check_refresh_selection(idx, layer.scores.cpu().numpy(), r["scores"], k, f"MLP refresh, step {s}")
         else:
             A, Y = O.mlp_delta(x, W1, B1, W2, idx, A, Y, 128)
         ratio, _ = assert_parity(out, Y, f"MLP output, step {s}", bf16_out=True)
@@ -82,8 +106,14 @@ def run_attn_loop(T, h, permille, seed=4):
         q, k, v = (np.ascontiguousarray(O.bf16_decode(chains[n][s]).transpose(1, 0, 2)) for n in ("q", "k", "v"))
         if sched.is_dense(s):
             r = O.attn_refresh(q, k, v, scale, 128, kk)
+            idx = layer.idx.cpu().numpy()
+            nb = idx.shape[1]
+            check_refresh_selection(idx.reshape(h * nb, kk), layer.scores.cpu().numpy(), r["mass"], kk,
+                                    f"attention refresh, step {s}")
+            m_c, l_c, acc_c = (r["m_c"], r["l_c"], r["acc_c"]) if np.array_equal(idx, r["idx"]) else \
+                O.complement_partial(q, k, v, idx, scale, 128)
             f = lambda a: O.f32(a).astype(np.float64)  # the partial is stored as fp32
-            cache, ref = (r["idx"], f(r["m_c"]), f(r["l_c"]), f(r["acc_c"])), r["O"]
+            cache, ref = (idx, f(m_c), f(l_c), f(acc_c)), r["O"]
         else:
             ref = O.attn_delta(q, k, v, *cache, scale, 128)
         ratio, _ = assert_parity(out, ref, f"attention output, step {s}", bf16_out=True)

@@ -10,7 +10,7 @@ import pytest
 
 import oracle as O
 from dynamic_column_sparse_b200 import synth
-from helpers import (assert_bf16_storage, assert_parity, bits_of, dev_bf16, dev_f32, f64_of, f64_of_bf16, heads_first, to_block_major,
+from helpers import (assert_bf16_storage, check_selection, assert_parity, bits_of, dev_bf16, dev_f32, f64_of, f64_of_bf16, heads_first, to_block_major,
                      to_token_major)
 
 pytestmark = pytest.mark.gpu
@@ -21,26 +21,6 @@ def cm():
     from dynamic_column_sparse_b200 import chipmunk
     chipmunk.load_library()
     return chipmunk
-
-
-def check_selection(idx, ref_scores, k, band):
-    """idx rows: strictly ascending, k distinct; every kept score >= every dropped score - band * scale."""
-    rows, n = ref_scores.shape
-    assert idx.shape == (rows, k)
-    same = 0
-    ref_idx = O.topk_cols(O.f32(ref_scores), k)
-    for r in range(rows):
-        sel = idx[r]
-        assert np.all(np.diff(sel) > 0) and sel.min() >= 0 and sel.max() < n
-        if np.array_equal(sel, ref_idx[r]):
-            same += 1
-            continue
-        mask = np.zeros(n, dtype=bool)
-        mask[sel] = True
-        scale = max(np.abs(ref_scores[r]).max(), 1e-30)
-        if k and k < n:
-            assert ref_scores[r][mask].min() >= ref_scores[r][~mask].max() - band * scale, f"row {r}"
-    return same
 
 
 @pytest.mark.parametrize("T,D,H,Bt,permille,first", [

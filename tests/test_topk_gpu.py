@@ -54,3 +54,34 @@ def test_topk_tiny_rows(cm):
         for k in range(0, n + 1, max(1, n // 3)):
             got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
             np.testing.assert_array_equal(got, O.topk_cols(s, k))
+
+
+@pytest.mark.parametrize("rows,n,k", [
+    (9, 45001, 3000),     # n not a multiple of 4: rows alternate between 16-byte aligned and not
+    (5, 118800, 8316),    # HunyuanVideo attention row
+    (3, 60000, 59999),
+    (3, 50000, 1),
+    (4, 50000, 30000),    # more candidates than the shared-memory buffer holds
+])
+def test_topk_long_rows(cm, rows, n, k):
+    s = synth.score_rows(11, rows, n, ties=True)
+    got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
+    np.testing.assert_array_equal(got, O.topk_cols(s, k))
+
+
+def test_topk_long_special_values(cm):
+    n = 50000
+    rows = []
+    rows.append(np.full(n, 0.5, dtype=np.float32))                               # all equal
+    r = np.zeros(n, dtype=np.float32); r[::3] = -0.0; r[5::7] = 1e-30; rows.append(r)
+    r = synth.score_rows(13, 1, n)[0] - 1.0; r[[0, 17, n - 1]] = np.inf; r[[3, 9]] = -np.inf; rows.append(r)
+    r = np.round(synth.score_rows(14, 1, n)[0] * 2) / 2; rows.append(r.astype(np.float32))   # few distinct values
+    # 20000 distinct values inside one 12-bit key bucket ([1, 1.125)) above 30000 small ones
+    r = synth.score_rows(15, 1, n)[0] * 1e-3
+    r[::5] = 1.0 + 0.1 * synth.uniform_f64(15, 99, (n + 4) // 5)[: len(r[::5])]
+    r[1::5] = 1.0 + 0.1 * synth.uniform_f64(16, 99, len(r[1::5]))
+    rows.append(r.astype(np.float32))
+    s = np.stack(rows).astype(np.float32)
+    for k in (1, 100, 4000, 19999, 20000, 20001, 49999):
+        got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
+        np.testing.assert_array_equal(got, O.topk_cols(s, k), err_msg=f"k={k}")
