@@ -53,3 +53,63 @@ def test_reference_arm_other_ranks_exit_without_work():
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def _lonely_worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    try:
+        dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=3))
+        out[rank] = "joined"
+        dist.destroy_process_group()
+    except Exception as e:  # the rendezvous ends with an error, not a hang
+        out[rank] = type(e).__name__
+
+
+def test_rank_that_never_joins_ends_in_a_bounded_error():
+    import time
+
+    import torch.multiprocessing as mp
+    port = _free_port()
+    t0 = time.time()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_lonely_worker, args=(2, port, out), nprocs=1, start_method="spawn", join=True)
+        res = dict(out)
+    assert res[0] != "joined"
+    assert time.time() - t0 < 60
+
+
+def _dying_worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left before the step's collective"
+        os._exit(3)  # the rank dies between steps, with nothing in flight
+    try:
+        bench.max_over_ranks(1.0)
+        out[rank] = "collective completed"
+    except Exception as e:
+        out[rank] = type(e).__name__
+
+
+def test_rank_that_dies_is_seen_by_the_other_rank():
+    import torch.multiprocessing as mp
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        ctx = mp.start_processes(_dying_worker, args=(2, port, out), nprocs=2, start_method="spawn", join=False)
+        for p in ctx.processes:
+            p.join(timeout=60)
+        codes = [p.exitcode for p in ctx.processes]
+        res = dict(out)
+    assert codes[1] == 3
+    assert res[1] == "left before the step's collective"
+    assert res.get(0) not in (None, "collective completed")
