@@ -443,7 +443,8 @@ def run_gpu(args):
         "clocks": clocks,
     }
     if world == 1 and not args.no_rows:
-        res["rows"] = extra_rows(L, w, peaks, flush, torch, cm)
+        groups = set(ROW_GROUPS) if args.rows == "all" else set(args.rows.split(","))
+        res["rows"] = extra_rows(L, w, peaks, flush, torch, cm, groups)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         smp = OracleSample(w)
         us = statistics.median([smp.time_step() for _ in range(3)])
@@ -459,7 +460,30 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def extra_rows(L, w, peaks, flush, torch, cm):
+def step_rows(Lx, w, reps, flush, torch):
+    """Per-kernel device time and useful TFLOP/s of one sparse step of layer Lx."""
+    T, D, H, h, d = w["T"], w["D"], w["H"], w["heads"], w["d"]
+    out = {"T": T, "mlp_k": Lx.kc, "attn_k": Lx.kk}
+    flops = {"mlp_up": 2 * T * D * Lx.kc, "mlp_down": 2 * T * D * Lx.kc, "attn_delta": 4 * T * Lx.kk * d * h}
+    total = 0.0
+    for name, fn in (("mlp_up", Lx.mlp_up), ("mlp_down", Lx.mlp_down), ("attn_delta", Lx.attn)):
+        it = [0]
+
+        def call():
+            it[0] += 1
+            fn(it[0])
+        call()
+        ms = time_events(call, reps, flush, torch)
+        total += ms
+        out[name] = {"us": round(ms * 1e3, 1), "tflops": round(flops[name] / (ms * 1e-3) / 1e12, 1)}
+    out["step_us"] = round(total * 1e3, 1)
+    return out
+
+
+ROW_GROUPS = ("topk", "cols", "refresh", "dense", "sweep", "workloads", "cublas")
+
+
+def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
     """The other rows of the hot path, timed with CUDA events (median of 10, L2 flushed)."""
     hbm = peaks["hbm_gbs"]
     rows = {}
@@ -470,7 +494,46 @@ def extra_rows(L, w, peaks, flush, torch, cm):
         return {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
                 "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
 
-    # a1: top-k over the layer's score rows, and over HunyuanVideo-length attention rows
+    if "topk" in groups:
+        topk_rows(L, w, rows, gbs, flush, torch, cm)
+    if "cols" in groups:
+        cols_rows(L, w, rows, gbs, flush, torch, cm)
+    q, k, v = L.qkv_prev
+    dense_mlp_f = 4 * T * D * H
+    dense_attn_f = 4 * T * T * w["d"] * h
+    if "refresh" in groups:
+        refresh_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f)
+    if "dense" in groups or "sweep" in groups:
+        dense_us = dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f)
+        if "sweep" in groups:
+            sweep_rows(L, w, rows, flush, torch, dense_us)
+    if "workloads" in groups:
+        # the same sparse step at two more workloads of the pages: FLUX.1-dev at 2304x1280
+        # (144 x 80 latent patches + 512 text tokens) and a HunyuanVideo layer (720x1280x129
+        # -> 33 x 45 x 80 = 118800 tokens, attention 93% sparse)
+        for name, extra, reps2 in (("flux_2304x1280_step", dict(T=144 * 80 + 512), 5),
+                                   ("hunyuan_step", dict(T=118800, attn_permille=70), 3)):
+            w2 = dict(w, **extra)
+            L2 = Layer(w2, L.dev, seed=99)
+            rows[name] = step_rows(L2, w2, reps2, flush, torch)
+            del L2
+            torch.cuda.empty_cache()
+    if "cublas" in groups:
+        xw = L.xs[0]
+        w1 = L.w1t.t()
+        ms_cub = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),
+                                                  L.w2), 5, flush, torch)
+        rows["dense_mlp_torch_context"] = {"us": round(ms_cub * 1e3, 1),
+                                           "note": "torch.matmul (cuBLAS) + GELU, context only"}
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    return rows
+
+
+def topk_rows(L, w, rows, gbs, flush, torch, cm):
+    """a1: top-k over the layer's score rows, and over HunyuanVideo-length attention rows."""
+    T, H, h = w["T"], w["H"], w["heads"]
+    reps = 10
     ms = time_events(lambda: cm.topk_cols(L.mlp_scores, L.kc, out=L.idx), reps, flush, torch)
     rows["topk_flux_mlp"] = dict(rows=L.nb, n=H, k=L.kc, **gbs(L.nb * (H + L.kc) * 4, ms))
     mass2 = L.mass.view(h * L.nb, T)
@@ -485,7 +548,13 @@ def extra_rows(L, w, peaks, flush, torch, cm):
     rows["topk_hunyuan_attn_rows"] = dict(rows=hr, n=hn, k=hk, note="2960 of 22296 HunyuanVideo mass rows",
                                           **gbs(hr * (hn + hk) * 4, ms))
     del hs, hidx
-    # a6: cache column gather / scatter (FLUX and HunyuanVideo-sized caches)
+
+
+def cols_rows(L, w, rows, gbs, flush, torch, cm):
+    """a6: cache column gather / scatter (FLUX and HunyuanVideo-sized caches)."""
+    H, Bt = w["H"], w["Bt"]
+    reps = 10
+    g = torch.Generator(device=L.dev).manual_seed(8)
     packed = torch.empty((L.nb, L.kc, Bt), dtype=torch.bfloat16, device=L.dev)
     nbytes = 2 * L.nb * L.kc * Bt * 2
     ms = time_events(lambda: cm.gather_cols(L.a_cache, L.idx, packed), reps, flush, torch)
@@ -504,19 +573,26 @@ def extra_rows(L, w, peaks, flush, torch, cm):
     ms = time_events(lambda: cm.scatter_cols(packed_h, idx_h, cache_h), 5, flush, torch)
     rows["scatter_hunyuan"] = gbs(nbytes, ms)
     del cache_h, idx_h, packed_h
-    # a5: dense refresh of the layer
+
+
+def refresh_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
+    """a5: dense refresh of the layer."""
+    Bt = w["Bt"]
     ms_mlp = time_events(lambda: cm.mlp_refresh(L.x_prev, L.w1t, L.b1, L.w2, L.b2, L.a_cache, L.y_cache, L.idx,
                                                 L.mlp_scores, L.out, Bt=Bt), 5, flush, torch)
     q, k, v = L.qkv_prev
     ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, L.mass,
                                                   scale=1 / math.sqrt(w["d"]), workspace=L.attn_ws), 5, flush, torch)
-    dense_mlp_f = 4 * T * D * H
-    dense_attn_f = 4 * T * T * w["d"] * h
     rows["refresh_mlp"] = {"us": round(ms_mlp * 1e3, 1),
                            "tflops": round(dense_mlp_f / (ms_mlp * 1e-3) / 1e12, 1)}
     rows["refresh_attn"] = {"us": round(ms_attn * 1e3, 1), "passes": "dense + mass + top-k + complement",
                             "tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1)}
-    # dense layer at the same shape with the same kernels (k = all columns, all keys)
+
+
+def dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
+    """The dense layer at the same shape with the same kernels (k = all columns, all keys)."""
+    T, H, h, Bt = w["T"], w["H"], w["heads"], w["Bt"]
+    q, k, v = L.qkv_prev
     idx_all = torch.arange(H, dtype=torch.int32, device=L.dev).repeat(L.nb, 1).contiguous()
     ws_all = torch.empty(cm.mlp_workspace_bytes(T, H, H, Bt), dtype=torch.uint8, device=L.dev)
     aidx_all = torch.arange(T, dtype=torch.int32, device=L.dev).repeat(h, L.nb, 1).contiguous()
@@ -530,10 +606,15 @@ def extra_rows(L, w, peaks, flush, torch, cm):
     rows["dense_layer_k_all"] = {"us": round((ms_dm + ms_da) * 1e3, 1), "mlp_us": round(ms_dm * 1e3, 1),
                                  "attn_us": round(ms_da * 1e3, 1),
                                  "tflops": round((dense_mlp_f + dense_attn_f) / ((ms_dm + ms_da) * 1e-3) / 1e12, 1)}
-    # multi-step schedule (10 steps, dense at 0 and 5) across sparsity levels, through the layer API
+    return (ms_dm + ms_da) * 1e3
+
+
+def sweep_rows(L, w, rows, flush, torch, dense_us):
+    """Multi-step schedule (10 steps, dense at 0 and 5) across sparsity levels, through the layer API."""
     from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaAttention, SparseDeltaMLP
+    T, h, Bt = w["T"], w["heads"], w["Bt"]
+    reps = 10
     sweep = {}
-    dense_us = (ms_dm + ms_da) * 1e3
     for mp, ap in ((500, 500), (300, 165), (150, 150), (70, 70)):
         mlp = SparseDeltaMLP(L.w1t, L.b1, L.w2, L.b2, T, Bt, mp)
         att = SparseDeltaAttention(T, h, L.dev, ap)
@@ -556,14 +637,6 @@ def extra_rows(L, w, peaks, flush, torch, cm):
             "speedup_vs_dense_k_all": round(dense_us / (ms_sp * 1e3), 2)}
         del mlp, att
     rows["loop_sweep"] = sweep
-    xw = L.xs[0]
-    w1 = L.w1t.t()
-    ms_cub = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),
-                                              L.w2), 5, flush, torch)
-    rows["dense_mlp_torch_context"] = {"us": round(ms_cub * 1e3, 1), "note": "torch.matmul (cuBLAS) + GELU, context only"}
-    torch.cuda.synchronize()
-    assert cm.read_device_status() == 0
-    return rows
 
 
 # ---------------------------------------------------------------- reference arm
@@ -601,6 +674,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the extra hot-path rows")
+    ap.add_argument("--rows", default="all",
+                    help="comma list of extra row groups: " + ",".join(ROW_GROUPS) + " (default: all)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
