@@ -480,7 +480,7 @@ def step_rows(Lx, w, reps, flush, torch):
     return out
 
 
-ROW_GROUPS = ("topk", "cols", "refresh", "dense", "sweep", "workloads", "cublas")
+ROW_GROUPS = ("topk", "cols", "refresh", "dense", "sweep", "compact", "workloads", "cublas")
 
 
 def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
@@ -507,6 +507,8 @@ def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
         dense_us = dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f)
         if "sweep" in groups:
             sweep_rows(L, w, rows, flush, torch, dense_us)
+    if "compact" in groups:
+        compact_rows(L, w, rows, flush, torch, hbm)
     if "workloads" in groups:
         # the same sparse step at two more workloads of the pages: FLUX.1-dev at 2304x1280
         # (144 x 80 latent patches + 512 text tokens) and a HunyuanVideo layer (720x1280x129
@@ -607,6 +609,30 @@ def dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
                                  "attn_us": round(ms_da * 1e3, 1),
                                  "tflops": round((dense_mlp_f + dense_attn_f) / ((ms_dm + ms_da) * 1e-3) / 1e12, 1)}
     return (ms_dm + ms_da) * 1e3
+
+
+def compact_rows(L, w, rows, flush, torch, hbm):
+    """Attention delta step with the complement cached as fp32 (m, l, acc) or compact (lse fp32, o_c bf16)."""
+    from dynamic_column_sparse_b200.layer import SparseDeltaAttention
+    T, h, d = w["T"], w["heads"], w["d"]
+    out = {}
+    for name, compact in (("partial_fp32", False), ("compact_lse_bf16", True)):
+        att = SparseDeltaAttention(T, h, L.dev, w["attn_permille"], compact=compact)
+        att.refresh(*L.qkv_prev)
+        it = [0]
+
+        def step():
+            it[0] += 1
+            att.step(*L.qkvs[it[0] % 2])
+        step()
+        ms = time_events(step, 10, flush, torch)
+        cache_bytes = h * T * (4 + d * 2) if compact else h * T * (8 + d * 4)
+        nbytes = 4 * T * h * d * 2 + cache_bytes + h * att.nb * att.k * 4
+        out[name] = {"us": round(ms * 1e3, 1), "tflops": round(4 * T * att.k * d * h / (ms * 1e-3) / 1e12, 1),
+                     "algorithmic_MB": round(nbytes / 1e6, 1),
+                     "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+        del att
+    rows["attn_delta_cache_forms"] = out
 
 
 def sweep_rows(L, w, rows, flush, torch, dense_us):

@@ -64,6 +64,7 @@ class AttnArgs(ctypes.Structure):
         ("q", ctypes.c_void_p), ("kk", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("idx", ctypes.c_void_p), ("m_c", ctypes.c_void_p), ("l_c", ctypes.c_void_p),
         ("acc_c", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("cache_format", ctypes.c_int32), ("lse_c", ctypes.c_void_p), ("o_c", ctypes.c_void_p),
     ]
 
 
@@ -250,19 +251,29 @@ def mlp_refresh(x, w1t, b1, w2, b2, a_cache, y_cache, idx, scores, out=None, Bt=
 
 # ------------------------------------------------------------------ attention
 
-def _attn_args(q, k, v, idx, m_c, l_c, acc_c, o, scale, kk):
+ATTN_CACHE_PARTIAL = 0
+ATTN_CACHE_COMPACT = 1
+
+
+def _attn_args(q, k, v, idx, m_c, l_c, acc_c, o, scale, kk, lse_c=None, o_c=None):
+    """Partial-form cache (m_c, l_c, acc_c) or, with lse_c / o_c given, the compact form."""
     T, h, d = q.shape
     nb = (T + 127) // 128
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _need(t, name, torch.bfloat16, (T, h, d))
     _need(idx, "idx", torch.int32, (h, nb, kk))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if lse_c is not None:
+        _need(lse_c, "lse_c", torch.float32, (h, T))
+        _need(o_c, "o_c", torch.bfloat16, (h, T, d))
+        return AttnArgs(T, h, d, 128, kk, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(),
+                        None, None, None, o.data_ptr(), ATTN_CACHE_COMPACT, lse_c.data_ptr(), o_c.data_ptr())
     _need(m_c, "m_c", torch.float32, (h, T))
     _need(l_c, "l_c", torch.float32, (h, T))
     _need(acc_c, "acc_c", torch.float32, (h, T, d))
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
     return AttnArgs(T, h, d, 128, kk, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(),
-                    m_c.data_ptr(), l_c.data_ptr(), acc_c.data_ptr(), o.data_ptr())
+                    m_c.data_ptr(), l_c.data_ptr(), acc_c.data_ptr(), o.data_ptr(), ATTN_CACHE_PARTIAL, None, None)
 
 
 def attn_delta(q, k, v, idx, m_c, l_c, acc_c, o, scale=None, stream=None):
@@ -273,10 +284,20 @@ def attn_delta(q, k, v, idx, m_c, l_c, acc_c, o, scale=None, stream=None):
     return o
 
 
-def attn_refresh(q, k, v, idx, m_c, l_c, acc_c, o, scores, scale=None, workspace=None, stream=None):
-    """Dense attention step: o, mass scores [h][nb][T], new selection idx and the complement cache."""
+def attn_delta_compact(q, k, v, idx, lse_c, o_c, o, scale=None, stream=None):
+    """Sparse attention step against the compact complement cache (lse_c fp32 [h][T], o_c bf16 [h][T][d])."""
     lib = load_library()
-    a = _attn_args(q, k, v, idx, m_c, l_c, acc_c, o, scale, idx.shape[2])
+    a = _attn_args(q, k, v, idx, None, None, None, o, scale, idx.shape[2], lse_c=lse_c, o_c=o_c)
+    _check(lib.chipmunk_attn_delta(ctypes.byref(a), None, 0, _stream(stream)))
+    return o
+
+
+def attn_refresh(q, k, v, idx, m_c, l_c, acc_c, o, scores, scale=None, workspace=None, stream=None, lse_c=None,
+                 o_c=None):
+    """Dense attention step: o, mass scores [h][nb][T], new selection idx and the complement cache
+    (partial form m_c, l_c, acc_c; or, with lse_c and o_c given and m_c, l_c, acc_c None, the compact form)."""
+    lib = load_library()
+    a = _attn_args(q, k, v, idx, m_c, l_c, acc_c, o, scale, idx.shape[2], lse_c=lse_c, o_c=o_c)
     T, h = q.shape[0], q.shape[1]
     _need(scores, "scores", torch.float32, (h, (T + 127) // 128, T))
     r = RefreshArgs(REFRESH_ATTN, 0, MlpArgs(), a, scores.data_ptr())

@@ -163,10 +163,15 @@ chipmunk_status check_attn(const chipmunk_attn_args *a, bool refresh) {
   if (!std::isfinite(a->scale)) return fail(CHIPMUNK_ERR_INVALID_ARG, "scale is not finite");
   if (refresh && cm::attn_smem_bytes(cm::kAttnComplement, a->T) > 227 * 1024)
     return fail(CHIPMUNK_ERR_SHAPE, "T=%lld too long for the complement pass", (long long)a->T);
-  const void *req[] = {a->q, a->kk, a->v, a->m_c, a->l_c, a->acc_c, a->o, a->idx};
-  const char *names[] = {"q", "kk", "v", "m_c", "l_c", "acc_c", "o", "idx"};
-  for (int i = 0; i < 8; ++i) {
-    if (req[i] == nullptr && !(i == 7 && !refresh && a->k == 0))
+  if (a->cache_format != CHIPMUNK_ATTN_CACHE_PARTIAL && a->cache_format != CHIPMUNK_ATTN_CACHE_COMPACT)
+    return fail(CHIPMUNK_ERR_INVALID_ARG, "cache_format=%d unknown", a->cache_format);
+  const bool compact = a->cache_format == CHIPMUNK_ATTN_CACHE_COMPACT;
+  const void *req[] = {a->q, a->kk, a->v, a->o, a->idx, compact ? static_cast<const void *>(a->lse_c) : a->m_c,
+                       compact ? a->o_c : static_cast<const void *>(a->l_c), compact ? nullptr : a->acc_c};
+  const char *names[] = {"q", "kk", "v", "o", "idx", compact ? "lse_c" : "m_c", compact ? "o_c" : "l_c", "acc_c"};
+  const int nreq = compact ? 7 : 8;
+  for (int i = 0; i < nreq; ++i) {
+    if (req[i] == nullptr && !(i == 4 && !refresh && a->k == 0))
       return fail(CHIPMUNK_ERR_INVALID_ARG, "%s is NULL", names[i]);
     if (req[i] != nullptr && !aligned16(req[i])) return fail(CHIPMUNK_ERR_ALIGNMENT, "%s is not 16-byte aligned", names[i]);
   }
@@ -314,7 +319,8 @@ chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, void *ws, size_
   CM_CHECK(map2d(&tm_v, a->v, a->T, cols, 64, 128, "v"));
   cm::AttnParams p{int(a->T), a->h, int(nb), a->k, a->scale * 1.4426950408889634f,
                    static_cast<const uint16_t *>(a->kk), static_cast<const uint16_t *>(a->v), a->idx, a->m_c,
-                   a->l_c, a->acc_c, static_cast<uint16_t *>(a->o), nullptr, status};
+                   a->l_c, a->acc_c, static_cast<uint16_t *>(a->o), nullptr, status,
+                   a->cache_format == CHIPMUNK_ATTN_CACHE_COMPACT, a->lse_c, static_cast<uint16_t *>(a->o_c)};
   CM_CUDA(cm::launch_attn(cm::kAttnDelta, p, tm_q, tm_k, tm_v, s), "attention delta launch");
   return CHIPMUNK_OK;
 }
@@ -368,7 +374,8 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
     const float sl2 = a->scale * 1.4426950408889634f;
     cm::AttnParams dense{int(a->T), a->h, int(nb), a->k, sl2, static_cast<const uint16_t *>(a->kk),
                          static_cast<const uint16_t *>(a->v), a->idx, a->m_c, a->l_c, a->acc_c,
-                         static_cast<uint16_t *>(a->o), lse, status};
+                         static_cast<uint16_t *>(a->o), lse, status,
+                         a->cache_format == CHIPMUNK_ATTN_CACHE_COMPACT, a->lse_c, static_cast<uint16_t *>(a->o_c)};
     CM_CUDA(cm::launch_attn(cm::kAttnDense, dense, tm_q, tm_k, tm_v, s), "attention refresh dense launch");
     cm::MassParams mp{int(a->T), a->h, int(nb), sl2, lse, r->scores, status};
     CM_CUDA(cm::launch_attn_mass(mp, tm_q, tm_k, s), "attention mass launch");

@@ -236,7 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (MODE == kAttnDelta && pw == 1 && lane == 0) {
         // the merge epilogue of this tile reads its rows of the complement accumulator
         const int nrows = min(128, T - b * 128);
-        prefetch_l2_bulk(p.acc_c + (static_cast<size_t>(hh) * T + b * 128) * 128, static_cast<uint32_t>(nrows) * 512u);
+        const size_t row0 = (static_cast<size_t>(hh) * T + b * 128) * 128;
+        if (p.compact)
+          prefetch_l2_bulk(p.o_c + row0, static_cast<uint32_t>(nrows) * 256u);
+        else
+          prefetch_l2_bulk(p.acc_c + row0, static_cast<uint32_t>(nrows) * 512u);
       }
       for (int i = 0; i <= nchunks; ++i) {
         if (i < nchunks && !load_k(g0 + i, i, hh)) {
@@ -355,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t row = static_cast<size_t>(hh) * T + gi;
       float mc = 0.f, lc = 0.f;
       if (MODE == kAttnDelta && gi < T) {
-        mc = p.m_c[row];
-        lc = p.l_c[row];
+        // compact cache: l_c e^(m_c) = e^(lse_c), so lse_c takes m_c's place with l_c = 1
+        mc = p.compact ? p.lse_c[row] : p.m_c[row];
+        lc = p.compact ? 1.f : p.l_c[row];
       }
       float m_used = -INFINITY, l = 0.f;   // m_used in log2 units of the scaled logits
       for (int i = 0; i < nchunks; ++i) {
@@ -464,12 +469,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += xs[(half ^ 1) * 128 + r];
       // complement accumulator row, this half's 64 dimensions: the first 32 are
       // loaded while P V of the last chunk runs, the rest (already pulled into
-      // L2 by the producers at the start of the tile) when they are merged
-      const float4 *acg = reinterpret_cast<const float4 *>(p.acc_c + row * 128 + half * 64);
+      // L2 by the producers at the start of the tile) when they are merged.
+      // The compact cache holds them as bf16: acv[0..3] then carry the raw
+      // 16-byte words of the first 32.
+      const bool compact = p.compact != 0;
+      const float4 *acg = compact ? nullptr : reinterpret_cast<const float4 *>(p.acc_c + row * 128 + half * 64);
+      const uint4 *ocg = compact ? reinterpret_cast<const uint4 *>(p.o_c + row * 128 + half * 64) : nullptr;
       float4 acv[8];
       if (MODE == kAttnDelta && gi < T) {
+        if (compact) {
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) acv[e4] = acg[e4];
+          for (int e = 0; e < 4; ++e) {
+            const uint4 u = ocg[e];
+            acv[e] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+          }
+        } else {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) acv[e4] = acg[e4];
+        }
       }
       if (nchunks > 0) {
         if (!wait_warp(&o_full[ob], (tl >> 1) & 1, p.status, abort_flag)) break;
@@ -484,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ws = (m2 == -INFINITY) ? 0.f : exp2_approx(m2 - M);
         const float L = lc * wc + l * ws;
         inv = L > 0.f ? 1.f / L : 0.f;
-      } else if (MODE == kAttnDense) {
+      } else if (MODE == kAttnDense || compact) {
         inv = l > 0.f ? 1.f / l : 0.f;
       }
       // O of this half in two groups of 32 dimensions
@@ -507,13 +524,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
 #pragma unroll
             for (int e8 = 0; e8 < 4; ++e8) {
-              const float4 a0 = c == 0 ? acv[2 * e8] : acg[8 + 2 * e8];
-              const float4 a1 = c == 0 ? acv[2 * e8 + 1] : acg[9 + 2 * e8];
+              float av[8];  // complement accumulator (partial) or normalised output (compact), dims d0 + 8 e8 ..
+              if (compact) {
+                const uint4 u = c == 0 ? make_uint4(__float_as_uint(acv[e8].x), __float_as_uint(acv[e8].y),
+                                                    __float_as_uint(acv[e8].z), __float_as_uint(acv[e8].w))
+                                       : ocg[4 + e8];
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  av[2 * j] = __uint_as_float(w4[j] << 16);
+                  av[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
+                }
+              } else {
+                const float4 a0 = c == 0 ? acv[2 * e8] : acg[8 + 2 * e8];
+                const float4 a1 = c == 0 ? acv[2 * e8 + 1] : acg[9 + 2 * e8];
+                av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w;
+                av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
+              }
               const float *oa = ov + 8 * e8;
-              orow[e8] = make_uint4(cvt_bf16x2((a0.x * wc + oa[0] * ws) * inv, (a0.y * wc + oa[1] * ws) * inv),
-                                    cvt_bf16x2((a0.z * wc + oa[2] * ws) * inv, (a0.w * wc + oa[3] * ws) * inv),
-                                    cvt_bf16x2((a1.x * wc + oa[4] * ws) * inv, (a1.y * wc + oa[5] * ws) * inv),
-                                    cvt_bf16x2((a1.z * wc + oa[6] * ws) * inv, (a1.w * wc + oa[7] * ws) * inv));
+              orow[e8] = make_uint4(cvt_bf16x2((av[0] * wc + oa[0] * ws) * inv, (av[1] * wc + oa[1] * ws) * inv),
+                                    cvt_bf16x2((av[2] * wc + oa[2] * ws) * inv, (av[3] * wc + oa[3] * ws) * inv),
+                                    cvt_bf16x2((av[4] * wc + oa[4] * ws) * inv, (av[5] * wc + oa[5] * ws) * inv),
+                                    cvt_bf16x2((av[6] * wc + oa[6] * ws) * inv, (av[7] * wc + oa[7] * ws) * inv));
             }
           } else if (MODE == kAttnDense) {
             uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
@@ -522,6 +554,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float *oa = ov + 8 * e8;
               orow[e8] = make_uint4(cvt_bf16x2(oa[0] * inv, oa[1] * inv), cvt_bf16x2(oa[2] * inv, oa[3] * inv),
                                     cvt_bf16x2(oa[4] * inv, oa[5] * inv), cvt_bf16x2(oa[6] * inv, oa[7] * inv));
+            }
+          } else if (compact) {
+            uint4 *oc = reinterpret_cast<uint4 *>(p.o_c + row * 128 + d0);
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) {
+              const float *oa = ov + 8 * e8;
+              oc[e8] = make_uint4(cvt_bf16x2(oa[0] * inv, oa[1] * inv), cvt_bf16x2(oa[2] * inv, oa[3] * inv),
+                                  cvt_bf16x2(oa[4] * inv, oa[5] * inv), cvt_bf16x2(oa[6] * inv, oa[7] * inv));
             }
           } else {
             float4 *ac = reinterpret_cast<float4 *>(p.acc_c + row * 128 + d0);
@@ -534,6 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (gi < T && half == 0) {
         if (MODE == kAttnDense) {
           p.lse[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
+        } else if (MODE == kAttnComplement && compact) {
+          p.lse_c[row] = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
         } else if (MODE == kAttnComplement) {
           p.m_c[row] = (m2 == -INFINITY) ? -INFINITY : m2 * kLn2;
           p.l_c[row] = l;

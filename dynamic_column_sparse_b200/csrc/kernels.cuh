@@ -74,10 +74,13 @@ struct AttnParams {
   float scale_log2;       // logit scale * log2(e)
   const uint16_t *k_ptr, *v_ptr;  // [T][h][128] (key rows gathered on a sparse step)
   const int32_t *idx;     // [h][nb][k]
-  float *m_c, *l_c, *acc_c;  // [h][T], [h][T], [h][T][128]
+  float *m_c, *l_c, *acc_c;  // [h][T], [h][T], [h][T][128] (partial-form complement cache)
   uint16_t *o;            // [T][h][128]
   float *lse;             // [h][T] (dense)
   int *status;
+  int compact;            // complement cache as lse_c [h][T] fp32 and o_c [h][T][128] bf16
+  float *lse_c;
+  uint16_t *o_c;
 };
 // tm_q: tile map over Q [T][h*128] (box 64 x 128). tm_k / tm_v: gather4 maps
 // (sparse step) or tile maps (dense, complement) over K, V [T][h*128].

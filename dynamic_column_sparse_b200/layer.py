@@ -68,10 +68,13 @@ class SparseDeltaAttention:
     """Attention ``softmax(scale q k^T) v`` per head with a cached complement partial.
 
     ``q, k, v`` are [T][h][128] bf16. ``density_permille`` is the kept
-    fraction of keys per (head, 128-query block).
+    fraction of keys per (head, 128-query block). With ``compact`` the
+    complement is cached as ``lse_c`` (fp32) and the normalised ``o_c`` (bf16)
+    instead of ``m_c``, ``l_c``, ``acc_c`` (fp32): half the bytes.
     """
 
-    def __init__(self, T: int, h: int, device, density_permille: int = 165, scale: float | None = None):
+    def __init__(self, T: int, h: int, device, density_permille: int = 165, scale: float | None = None,
+                 compact: bool = False):
         d = 128
         self.T, self.h, self.d = T, h, d
         self.nb = (T + 127) // 128
@@ -79,9 +82,16 @@ class SparseDeltaAttention:
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         f32 = torch.float32
         self.idx = torch.zeros((h, self.nb, self.k), dtype=torch.int32, device=device)
-        self.m_c = torch.empty((h, T), dtype=f32, device=device)
-        self.l_c = torch.empty((h, T), dtype=f32, device=device)
-        self.acc_c = torch.empty((h, T, d), dtype=f32, device=device)
+        self.compact = compact
+        if compact:
+            self.lse_c = torch.empty((h, T), dtype=f32, device=device)
+            self.o_c = torch.empty((h, T, d), dtype=torch.bfloat16, device=device)
+            self.m_c = self.l_c = self.acc_c = None
+        else:
+            self.m_c = torch.empty((h, T), dtype=f32, device=device)
+            self.l_c = torch.empty((h, T), dtype=f32, device=device)
+            self.acc_c = torch.empty((h, T, d), dtype=f32, device=device)
+            self.lse_c = self.o_c = None
         self.o = torch.empty((T, h, d), dtype=torch.bfloat16, device=device)
         self.scores = torch.empty((h, self.nb, T), dtype=f32, device=device)
         self.workspace = torch.empty(h * T * 4, dtype=torch.uint8, device=device)
@@ -90,7 +100,7 @@ class SparseDeltaAttention:
     def refresh(self, q, k, v, stream=None):
         """Dense step: output, attention mass, new key selection, complement cache."""
         cm.attn_refresh(q, k, v, self.idx, self.m_c, self.l_c, self.acc_c, self.o, self.scores, scale=self.scale,
-                        workspace=self.workspace, stream=stream)
+                        workspace=self.workspace, stream=stream, lse_c=self.lse_c, o_c=self.o_c)
         self.has_cache = True
         return self.o
 
@@ -98,7 +108,10 @@ class SparseDeltaAttention:
         """Sparse step: selected keys with the current q, k, v, merged with the cached complement."""
         if not self.has_cache:
             raise RuntimeError("a sparse step needs a refresh first")
-        cm.attn_delta(q, k, v, self.idx, self.m_c, self.l_c, self.acc_c, self.o, scale=self.scale, stream=stream)
+        if self.compact:
+            cm.attn_delta_compact(q, k, v, self.idx, self.lse_c, self.o_c, self.o, scale=self.scale, stream=stream)
+        else:
+            cm.attn_delta(q, k, v, self.idx, self.m_c, self.l_c, self.acc_c, self.o, scale=self.scale, stream=stream)
         return self.o
 
 

@@ -114,8 +114,23 @@ typedef struct chipmunk_mlp_args {
  *   acc_c   [h][T][d]   fp32   m = max logit, l = sum exp(s - m),
  *                              acc = sum exp(s - m) v; an empty complement is
  *                              m = -inf, l = 0, acc = 0
+ *                              (cache_format CHIPMUNK_ATTN_CACHE_PARTIAL)
  *   o       [T][h][d]   bf16   output
+ *   cache_format               CHIPMUNK_ATTN_CACHE_PARTIAL (0): the complement
+ *                              is cached as m_c, l_c, acc_c above; lse_c and
+ *                              o_c are not used (may be NULL).
+ *                              CHIPMUNK_ATTN_CACHE_COMPACT (1): it is cached as
+ *   lse_c   [h][T]      fp32   lse = m + ln l (natural log, of the scaled
+ *                              logits; -inf for an empty complement) and
+ *   o_c     [h][T][d]   bf16   o = acc / l (0 for an empty complement); m_c,
+ *                              l_c, acc_c are not used (may be NULL). Same
+ *                              state in half the bytes of acc: o_c is rounded
+ *                              to bf16. (The post caches the partial state;
+ *                              this log-sum-exp encoding of it is the
+ *                              library's own.)
  */
+#define CHIPMUNK_ATTN_CACHE_PARTIAL 0
+#define CHIPMUNK_ATTN_CACHE_COMPACT 1
 typedef struct chipmunk_attn_args {
   int64_t T;
   int32_t h, d, Bt, k;
@@ -124,6 +139,9 @@ typedef struct chipmunk_attn_args {
   int32_t *idx;
   float *m_c, *l_c, *acc_c;
   void *o;
+  int32_t cache_format;
+  float *lse_c;
+  void *o_c;
 } chipmunk_attn_args;
 
 #define CHIPMUNK_REFRESH_MLP  0
@@ -140,8 +158,9 @@ typedef struct chipmunk_attn_args {
  *   kind == CHIPMUNK_REFRESH_ATTN: reads attn.{q,kk,v}; writes attn.o (dense
  *     attention), scores [h][nb][T] (fp32 attention mass: per query block
  *     the column sums of the softmax probabilities), attn.idx (top attn.k keys
- *     of each mass row) and attn.{m_c,l_c,acc_c} (the partial state of every
- *     query over the keys its block did not select).
+ *     of each mass row) and the complement cache of every query over the
+ *     keys its block did not select, in attn.cache_format: attn.{m_c,l_c,acc_c}
+ *     or attn.{lse_c,o_c}.
  */
 typedef struct chipmunk_refresh_args {
   int32_t kind;
@@ -230,6 +249,9 @@ CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args 
  * block the selected keys idx[h][b] are attended with the current q, kk, v by
  * online softmax and merged with the cached complement partial:
  *   M = max(m_c, m_s);  o = (acc_c e^(m_c-M) + acc_s e^(m_s-M)) / (l_c e^(m_c-M) + l_s e^(m_s-M)).
+ * With the compact cache (cache_format 1) the complement enters as
+ * l_c e^(m_c) = e^(lse_c) and acc_c e^(m_c) = o_c e^(lse_c):
+ *   M = max(lse_c, m_s);  o = (o_c e^(lse_c-M) + acc_s e^(m_s-M)) / (e^(lse_c-M) + l_s e^(m_s-M)).
  * Rows where nothing contributes (l = 0 on both sides) get 0. The cache is
  * read only. Needs no workspace.
  */

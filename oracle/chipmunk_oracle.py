@@ -232,6 +232,38 @@ def attn_delta(q, k, v, idx, m_c, l_c, acc_c, scale, Bt):
     return O
 
 
+def compact_partial(m, l, acc):
+    """The same partial state in log-sum-exp form: ``lse = m + ln l`` and the
+    normalised output ``o = acc / l``; an empty partial (l = 0) gives
+    ``(-inf, 0)``. Since ``e^lse = l e^m`` and ``o e^lse = acc e^m``, a merge
+    needs nothing else. (A denser encoding of the cached partial of the post's
+    attention step; the encoding is this library's.)
+    """
+    l = np.asarray(l, dtype=np.float64)
+    safe = np.where(l > 0, l, 1.0)
+    lse = np.where(l > 0, np.asarray(m, dtype=np.float64) + np.log(safe), NEG_INF)
+    o = np.where((l > 0)[..., None], np.asarray(acc, dtype=np.float64) / safe[..., None], 0.0)
+    return lse, o
+
+
+def attn_delta_compact(q, k, v, idx, lse_c, o_c, scale, Bt):
+    """Sparse attention step against a complement cached as ``(lse_c, o_c)``.
+
+    The cached complement enters the online-softmax merge as the partial
+    ``(lse_c, 1, o_c)``: relative to a shared maximum M its weight is
+    ``e^(lse_c - M)`` and its numerator ``o_c e^(lse_c - M)``. Returns O [h][T][d].
+    """
+    h, T, d = q.shape
+    O = np.zeros((h, T, d))
+    for hh in range(h):
+        for b, r0, r1 in blocks(T, Bt):
+            S = np.asarray(idx[hh][b], dtype=np.int64)
+            sel = attn_partial(q[hh, r0:r1], k[hh, S], v[hh, S], scale)
+            cached = (lse_c[hh, r0:r1], np.ones(r1 - r0), o_c[hh, r0:r1])
+            O[hh, r0:r1] = finish(merge_partials(cached, sel))
+    return O
+
+
 def dense_attention(q, k, v, scale):
     """``softmax(scale q k^T) v`` per head (post: "Attention" equation) and the row log-sum-exp."""
     h, T, d = q.shape

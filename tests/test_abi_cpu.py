@@ -37,13 +37,34 @@ def test_library_exports_every_declared_symbol(cm):
     assert set(cm.EXPORTS) <= set(declared_functions())
 
 
-def test_struct_layouts_match_the_header(cm):
-    # int64 x3 + int32 x2 + 9 pointers
-    assert ctypes.sizeof(cm.MlpArgs) == 24 + 8 + 9 * 8
-    # int64 + int32 x4 + float + pad + 8 pointers
-    assert ctypes.sizeof(cm.AttnArgs) == 8 + 16 + 4 + 4 + 8 * 8
-    assert cm.RefreshArgs.mlp.offset == 8
-    assert cm.RefreshArgs.scores.offset == 8 + ctypes.sizeof(cm.MlpArgs) + ctypes.sizeof(cm.AttnArgs)
+def test_struct_layouts_match_the_header(cm, tmp_path):
+    """Every field of the ctypes structs sits where a C compiler puts it for include/chipmunk.h."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    structs = {"chipmunk_mlp_args": cm.MlpArgs, "chipmunk_attn_args": cm.AttnArgs,
+               "chipmunk_refresh_args": cm.RefreshArgs}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", "#include \"chipmunk.h\"", "int main(void) {"]
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run([gcc, "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        cname, field, val = line.split()
+        got[(cname, field)] = int(val)
+    for cname, py in structs.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
 
 
 def test_version_and_status_strings(cm):

@@ -76,3 +76,48 @@ def test_attn_delta_fresh_cache_is_dense(cm):
     got = run_gpu(cm, c, c["idx"])
     dense, _ = O.dense_attention(c["q"], c["k"], c["v"], c["scale"])
     assert_parity(got, dense, "o vs dense attention", bf16_out=True)
+
+
+# --------------------------------------------------------------- compact complement cache
+
+def compact_of(c):
+    """The case's complement partial in compact form, at storage precision (lse fp32, o_c bf16 bits)."""
+    lse, oc = O.compact_partial(c["m_c"].astype(np.float64), c["l_c"].astype(np.float64), c["acc_c"].astype(np.float64))
+    return O.f32(lse), O.bf16_round(oc)
+
+
+def run_gpu_compact(cm, c, idx, lse32, oc_bits):
+    import torch
+    T, h, L = c["T"], c["h"], c["L"]
+    o = torch.empty((T, h, 128), dtype=torch.bfloat16, device="cuda")
+    cm.attn_delta_compact(dev_bf16(L["q"]), dev_bf16(L["k"]), dev_bf16(L["v"]), dev_i32(idx), dev_f32(lse32),
+                          dev_bf16(oc_bits), o, scale=c["scale"])
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    return heads_first(f64_of_bf16(o))
+
+
+@pytest.mark.parametrize("seed,T,h,permille", [
+    (1, 300, 2, 165),
+    (1, 700, 3, 400),
+    (0, 4352, 24, 165),   # FLUX layer
+])
+def test_attn_delta_compact_cache(cm, seed, T, h, permille):
+    c = attn_case(seed, T, h, permille, 0.03)
+    lse32, oc_bits = compact_of(c)
+    got = run_gpu_compact(cm, c, c["idx"], lse32, oc_bits)
+    ref = O.attn_delta_compact(c["q"], c["k"], c["v"], c["idx"], lse32.astype(np.float64), O.bf16_decode(oc_bits),
+                               c["scale"], 128)
+    assert_parity(got, ref, "o (compact cache)", bf16_out=True)
+
+
+def test_attn_delta_compact_cache_empty_sides(cm):
+    c = attn_case(1, 300, 2, 165, 0.03)
+    lse32, oc_bits = compact_of(c)
+    none = np.zeros((2, 3, 0), dtype=np.int32)
+    assert_parity(run_gpu_compact(cm, c, none, lse32, oc_bits), O.bf16_decode(oc_bits), "o = o_c", bf16_out=True)
+    allk = np.tile(np.arange(300, dtype=np.int32), (2, 3, 1))
+    empty_lse = np.full((2, 300), -np.inf, dtype=np.float32)
+    zeros = np.zeros((2, 300, 128), dtype=np.uint16)
+    dense, _ = O.dense_attention(c["q"], c["k"], c["v"], c["scale"])
+    assert_parity(run_gpu_compact(cm, c, allk, empty_lse, zeros), dense, "o vs dense attention", bf16_out=True)

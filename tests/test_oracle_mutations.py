@@ -153,6 +153,25 @@ def _bf16_truncate(x):
     return (f.view(np.uint32) >> 16).astype(np.uint16)
 
 
+def _compact_no_log(m, l, acc):
+    l = np.asarray(l, dtype=np.float64)
+    safe = np.where(l > 0, l, 1.0)
+    o = np.where((l > 0)[..., None], np.asarray(acc, dtype=np.float64) / safe[..., None], 0.0)
+    return np.where(l > 0, np.asarray(m, dtype=np.float64) + l, -np.inf), o
+
+
+def _delta_compact_unweighted(q, k, v, idx, lse_c, o_c, scale, Bt):
+    h, T, d = q.shape
+    out = np.zeros((h, T, d))
+    for hh in range(h):
+        for b, r0, r1 in OC.blocks(T, Bt):
+            S = np.asarray(idx[hh][b], dtype=np.int64)
+            sel = OC.attn_partial(q[hh, r0:r1], k[hh, S], v[hh, S], scale)
+            cached = (np.zeros(r1 - r0), np.ones(r1 - r0), o_c[hh, r0:r1])  # lse dropped from the weight
+            out[hh, r0:r1] = OC.finish(OC.merge_partials(cached, sel))
+    return out
+
+
 MUTATIONS = {
     "gelu_tanh: cubic term dropped": ("gelu_tanh", _gelu_no_cubic),
     "gelu_tanh: sign of tanh flipped": ("gelu_tanh", _gelu_sign),
@@ -168,6 +187,8 @@ MUTATIONS = {
     "complement_partial: selected keys kept": ("complement_partial", _complement_keeps_selected),
     "mlp_scores: absolute value dropped": ("mlp_scores", _scores_no_abs),
     "bf16_round: truncation instead of nearest-even": ("bf16_round", _bf16_truncate),
+    "compact_partial: log of l dropped": ("compact_partial", _compact_no_log),
+    "attn_delta_compact: cached weight e^lse dropped": ("attn_delta_compact", _delta_compact_unweighted),
 }
 
 

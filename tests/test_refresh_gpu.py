@@ -94,3 +94,39 @@ def test_attn_refresh(cm, T, h, permille):
     got_lse = np.concatenate([gm[hh, r0:r1] + np.log(gl[hh, r0:r1]) for hh, r0, r1 in rows])
     ref_lse = np.concatenate([ref["m_c"][hh, r0:r1] + np.log(ref["l_c"][hh, r0:r1]) for hh, r0, r1 in rows])
     assert np.max(np.abs(got_lse - ref_lse)) < 1e-3, "complement log-sum-exp"
+
+
+@pytest.mark.parametrize("T,h,permille", [(700, 2, 300), (4352, 24, 165)])
+def test_attn_refresh_compact_cache(cm, T, h, permille):
+    """The refresh writes the complement as lse_c (fp32) and o_c (bf16) when asked."""
+    import torch
+    L = synth.attn_layer(6, T, h, 128, 0.03)
+    hf = lambda a: np.ascontiguousarray(O.bf16_decode(a).transpose(1, 0, 2))
+    q, k, v = hf(L["q"]), hf(L["k"]), hf(L["v"])
+    scale = 1.0 / np.sqrt(128)
+    kk = O.k_from_density(T, permille)
+    nb = (T + 127) // 128
+    o = torch.empty((T, h, 128), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((h, nb, kk), dtype=torch.int32, device="cuda")
+    lse_c = torch.empty((h, T), dtype=torch.float32, device="cuda")
+    o_c = torch.empty((h, T, 128), dtype=torch.bfloat16, device="cuda")
+    scores = torch.empty((h, nb, T), dtype=torch.float32, device="cuda")
+    cm.attn_refresh(dev_bf16(L["q"]), dev_bf16(L["k"]), dev_bf16(L["v"]), idx, None, None, None, o, scores,
+                    scale=scale, lse_c=lse_c, o_c=o_c)
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    ref = O.attn_refresh(q, k, v, scale, 128, kk)
+    assert_parity(heads_first(f64_of_bf16(o)), ref["O"], "o", bf16_out=True)
+    g_idx = idx.cpu().numpy()
+    same = check_selection(g_idx.reshape(h * nb, kk), ref["mass"].reshape(h * nb, T), kk, band=2e-3)
+    assert same >= 0.9 * h * nb
+    ref_lse, ref_oc = O.compact_partial(ref["m_c"], ref["l_c"], ref["acc_c"])
+    got_lse, got_oc = f64_of(lse_c), f64_of_bf16(o_c)
+    rows = [(hh, r0, r1) for hh in range(h) for b, r0, r1 in O.blocks(T, 128)
+            if np.array_equal(g_idx[hh, b], ref["idx"][hh, b])]
+    cat = lambda a: np.concatenate([a[hh, r0:r1] for hh, r0, r1 in rows])
+    assert np.max(np.abs(cat(got_lse) - cat(ref_lse))) < 1e-3, "complement log-sum-exp"
+    # o_c is a normalised attention output over the complement (P enters the MMA as bf16, as for o):
+    # the bf16-output bar of o applies
+    assert_parity(cat(got_oc), cat(ref_oc), "complement o_c", bf16_out=True)
+
