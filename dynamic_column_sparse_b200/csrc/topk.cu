@@ -7,12 +7,15 @@
 //
 // Rows of up to kStagedMaxN scores are staged in shared memory once and run a
 // three-pass radix select (11 + 11 + 10 bits) there. Longer rows take two
-// vectorised passes over global memory: a 12-bit histogram finds the bucket
-// holding the k-th key, then every element at or above that bucket is copied
-// (key and index, in index order) into shared memory, where the remaining
-// 20 bits are resolved and the output is compacted. A row whose candidates do
-// not fit, or that is not 16-byte aligned, falls back to the general path that
-// re-reads the row from global memory for every radix pass.
+// vectorised passes over global memory (two rows in flight per SM): a 12-bit
+// histogram finds the bucket holding the k-th key, then every element at or
+// above that bucket is copied (key and index, in index order) into shared
+// memory, each warp appending its own segment of the row to its own region;
+// the remaining 20 bits are resolved and the output compacted there. If one
+// warp's region overflows while the row's candidates still fit, the regions
+// are laid end to end after a counting pass. A row whose candidates do not
+// fit at all, or that is not 16-byte aligned, falls back to the general path
+// that re-reads the row from global memory for every radix pass.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -25,7 +28,7 @@ constexpr int kMaxBins = 2048;
 constexpr int kItems = 8;             // consecutive elements per thread in the compaction
 constexpr int kStagedMaxN = 40960;    // 160 KB of keys in shared memory
 constexpr int kLongBins = 4096;       // first digit of the long-row path: the top 12 key bits
-constexpr int kLongCap = 24576;       // long-row candidates held in shared memory (192 KB)
+constexpr int kLongCap = 12288;       // long-row candidates held in shared memory (96 KB: two CTAs per SM)
 
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -204,6 +207,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
   __shared__ uint64_t warp_tot[kWarps + 1];
   __shared__ uint32_t s_digit, s_above;
   __shared__ uint32_t s_pref[kWarps + 1];  // start of warp w's candidates in the concatenated order
+  __shared__ uint32_t s_base[kWarps];      // where warp w's candidates sit in the buffer
   __shared__ int s_overflow;
   constexpr int kRegion = kLongCap / kWarps;
   constexpr int kUnroll = 8;
@@ -253,19 +257,27 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
     __syncthreads();
     select_digit(hist, kLongBins, k, warp_tot, s_digit, s_above);
     const uint32_t b1 = s_digit;
-    const int kk1 = k - static_cast<int>(s_above);  // keys to take from bucket b1
+    const int kk1 = k - static_cast<int>(s_above);   // keys to take from bucket b1
+    const uint32_t n_cand = s_above + hist[b1];       // keys in bucket b1 or above
     __syncthreads();
+    if (n_cand > static_cast<uint32_t>(kLongCap)) {
+      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
+      continue;
+    }
     // pass 2: warp w takes float4 elements [w seg, (w+1) seg) (the last warp also
     // the < 4 trailing scalars) and appends every key in bucket b1 or above,
-    // with its index, to its own region, in index order
-    {
-      const int seg = (n4 + kWarps - 1) / kWarps;
-      const int f_lo = min(warp * seg, n4), f_hi = min(f_lo + seg, n4);
-      uint32_t *wkey = ckey + warp * kRegion;
-      int32_t *widx = cidx + warp * kRegion;
+    // with its index, in index order, to its own region of the buffer
+    // (region w at s_base[w]). If a region overflows, every warp counts its
+    // candidates first, the regions are laid end to end, and the segments are
+    // read a second time.
+    const int seg = (n4 + kWarps - 1) / kWarps;
+    const int f_lo = min(warp * seg, n4), f_hi = min(f_lo + seg, n4);
+    // one pass over this warp's segment: counts (write false) or appends into
+    // wkey / widx up to cap entries; returns the count, sets over past cap
+    auto scan_segment = [&](bool write, uint32_t *wkey, int32_t *widx, uint32_t cap, bool &over) -> uint32_t {
       uint32_t wcount = 0;
-      bool over = false;
-      // appends this lane's flagged keys of one step (up to 4, elements base..base+3) in lane order
+      over = false;
+      // this lane's flagged keys of one step (up to 4, elements base..base+3), in lane order
       auto append = [&](const uint32_t *key, int base, int nvalid) {
         uint32_t flags = 0, cnt = 0;
 #pragma unroll
@@ -281,18 +293,20 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
           if (lane >= o) incl += t;
         }
         const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-        if (wcount + tot > static_cast<uint32_t>(kRegion)) {
-          over = true;  // warp-uniform
-          return;
-        }
-        uint32_t pos = wcount + incl - cnt;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (flags & (1u << c)) {
-            wkey[pos] = key[c];
-            widx[pos] = base + c;
-            ++pos;
+        if (write) {
+          if (wcount + tot > cap) {
+            over = true;  // warp-uniform
+            return;
           }
+          uint32_t pos = wcount + incl - cnt;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (flags & (1u << c)) {
+              wkey[pos] = key[c];
+              widx[pos] = base + c;
+              ++pos;
+            }
+        }
         wcount += tot;
       };
       for (int f0 = f_lo; f0 < f_hi && !over; f0 += kUnroll * 32) {
@@ -318,26 +332,40 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
           for (int c = 0; c < nt; ++c) key[c] = ordered_key(__ldg(src + 4 * n4 + c));
         append(key, 4 * n4, lane == 0 ? nt : 0);
       }
+      return wcount;
+    };
+    {
+      bool over;
+      const uint32_t wc = scan_segment(true, ckey + warp * kRegion, cidx + warp * kRegion, kRegion, over);
       if (lane == 0) {
-        warp_tot[warp] = wcount;
+        warp_tot[warp] = wc;
         if (over) s_overflow = 1;
       }
     }
     __syncthreads();
-    if (s_overflow) {
+    const bool contiguous = s_overflow != 0;
+    if (contiguous) {
+      bool over;
+      const uint32_t wc = scan_segment(false, nullptr, nullptr, 0, over);
+      if (lane == 0) warp_tot[warp] = wc;
       __syncthreads();
-      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
-      continue;
     }
     if (tid == 0) {
       uint32_t acc = 0;
       for (int w = 0; w < kWarps; ++w) {
         s_pref[w] = acc;
+        s_base[w] = contiguous ? acc : static_cast<uint32_t>(w * kRegion);
         acc += static_cast<uint32_t>(warp_tot[w]);
       }
       s_pref[kWarps] = acc;
     }
     __syncthreads();
+    if (contiguous) {
+      // the counts add up to n_cand <= kLongCap, so the regions laid end to end fit
+      bool over;
+      scan_segment(true, ckey + s_base[warp], cidx + s_base[warp], static_cast<uint32_t>(kLongCap), over);
+      __syncthreads();
+    }
     const int count = static_cast<int>(s_pref[kWarps]);
     // candidate L of the concatenated (index-ordered) list
     auto cand_at = [&](int L, uint32_t &key, int32_t &idx) {
@@ -345,7 +373,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
 #pragma unroll
       for (int step = kWarps / 2; step >= 1; step >>= 1)
         if (static_cast<uint32_t>(L) >= s_pref[w + step]) w += step;
-      const int j = w * kRegion + (L - static_cast<int>(s_pref[w]));
+      const int j = static_cast<int>(s_base[w]) + (L - static_cast<int>(s_pref[w]));
       key = ckey[j];
       idx = cidx[j];
     };
@@ -360,7 +388,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
       for (int w = 0; w < kWarps; ++w) {
         const int cw = static_cast<int>(s_pref[w + 1] - s_pref[w]);
         for (int j = tid; j < cw; j += kThreads) {
-          const uint32_t key = ckey[w * kRegion + j];
+          const uint32_t key = ckey[s_base[w] + j];
           if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
         }
       }
@@ -413,7 +441,7 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
     const int64_t grid = std::min<int64_t>(p.rows, static_cast<int64_t>(sms) * std::max(per_sm, 1));
     topk_kernel<true><<<static_cast<unsigned>(grid), kThreads, smem, s>>>(p);
   } else {
-    // one CTA per SM keeps every row being scanned resident in L2 between passes
+    // rows being scanned (two per SM) stay resident in L2 between the two passes
     const int smem = 2 * kLongCap * static_cast<int>(sizeof(uint32_t));
     static bool long_attr_set = false;
     if (!long_attr_set) {
@@ -421,7 +449,9 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       long_attr_set = true;
     }
-    const int64_t grid = std::min<int64_t>(p.rows, sms);
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_long_kernel, kThreads, smem);
+    const int64_t grid = std::min<int64_t>(p.rows, static_cast<int64_t>(sms) * std::max(per_sm, 1));
     topk_long_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(p);
   }
   return cudaGetLastError();

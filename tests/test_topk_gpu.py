@@ -85,3 +85,15 @@ def test_topk_long_special_values(cm):
     for k in (1, 100, 4000, 19999, 20000, 20001, 49999):
         got = cm.topk_cols(dev_f32(s), k).cpu().numpy()
         np.testing.assert_array_equal(got, O.topk_cols(s, k), err_msg=f"k={k}")
+
+
+def test_topk_long_rows_clustered_candidates(cm):
+    """The top scores crowd one part of the row: one warp's share of the candidates outgrows its
+    region while the row's total still fits (the candidates are then laid end to end)."""
+    rows, n, k = 4, 60000, 3000
+    s = synth.score_rows(17, rows, n, ties=True) * 1e-3
+    hot = synth.score_rows(18, rows, 4000, ties=True) + 1.0
+    s[:, 1000:5000] = hot                                 # the 3000 largest all sit in 4000 consecutive columns
+    s[2, 30000:34000] = hot[2]                            # and, on one row, in two such runs
+    got = cm.topk_cols(dev_f32(s.astype(np.float32)), k).cpu().numpy()
+    np.testing.assert_array_equal(got, O.topk_cols(s.astype(np.float32), k))
