@@ -2,17 +2,19 @@
 // plus the dense passes of the refresh (full attention with row log-sum-exp,
 // attention mass per query block, complement partial).
 //
-// One CTA per (head, 128-query block). Q arrives once by a tiled TMA load; K
-// and V stream in chunks of 128 keys through a two-stage ring: on a sparse
-// step the producer warps 5-7 gather the selected key rows with 16-byte
-// cp.async (one warp instruction = two whole 256-byte key rows), on the dense
-// passes one thread issues tiled TMA loads. Warp 4 issues the tcgen05 MMAs:
-// S = Q K^T into one of two TMEM buffers, then O_tmp = P V into a third.
-// Warps 0-3 run the online softmax, one query row per thread: they
-// read S from TMEM, write P (bf16) into a 128-byte-swizzled shared tile that is
-// the A operand of the next P V, and fold each O_tmp into a register
-// accumulator rescaled by the running max. S of chunk i+1 is computed while the
-// softmax of chunk i runs. Logits are kept in log2 units (scale * log2 e).
+// Persistent CTAs walk (head, 128-query block) tiles. Q arrives once per tile
+// by a tiled TMA load; K and V stream in chunks of 128 keys through two-stage
+// rings, K one chunk ahead of V: on a sparse step producer warps 9-11 gather
+// the selected key rows with 16-byte cp.async (one warp instruction = two
+// whole 256-byte key rows), on the dense passes one thread issues tiled TMA
+// loads. Warp 8 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
+// buffers, then O += P V into a TMEM accumulator (two, alternating between
+// tiles). Warps 0-7 run the online softmax, two warps per TMEM lane quadrant
+// (32 query rows), each on one 64-key half of S: both read the whole row to
+// take its maximum, exponentiate their half into P (bf16, a 128-byte-swizzled
+// shared tile, the A operand of the next P V) and rescale O in TMEM only when
+// the row maximum grows by more than 2^8. S of chunk i+1 is computed while
+// the softmax of chunk i runs. Logits are kept in log2 units (scale * log2 e).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -32,7 +34,7 @@ constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two
 constexpr float kRescaleLog2 = 8.0f;     // O and l are rescaled only when the row max grows by more than 2^8
 
 // Shared memory: Q | K[2] | V[2] | P | barriers | key-index ring [4][128] |
-// row-max exchange [2][2][128] | row-sum exchange [2][2][128] | key mask (complement pass).
+// row-sum exchange [2][2][128] | key mask (complement pass).
 struct AttnCfg {
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kTileBytes;
@@ -40,8 +42,7 @@ struct AttnCfg {
   static constexpr uint32_t kPOff = kVOff + 2 * kTileBytes;
   static constexpr uint32_t kBarOff = kPOff + kTileBytes;
   static constexpr uint32_t kIdxOff = kBarOff + 256;
-  static constexpr uint32_t kXmaxOff = kIdxOff + 4 * 128 * 4;
-  static constexpr uint32_t kXsumOff = kXmaxOff + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kXsumOff = kIdxOff + 4 * 128 * 4;
   static constexpr uint32_t kMaskOff = kXsumOff + 2 * 2 * 128 * 4;
 };
 
@@ -86,7 +87,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [4][128] selected keys of chunk g at g & 3
-  float *xmax = reinterpret_cast<float *>(smem + C::kXmaxOff);   // [2][2][128] partial row maxima
   float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
   uint32_t *mask = reinterpret_cast<uint32_t *>(smem + C::kMaskOff);
 
@@ -371,6 +371,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        // keys of the chunk that take part, per 32-key group q32 (0..3): bit e = key i*128 + 32 q32 + e
+        auto live_bits = [&](int q32) -> uint32_t {
+          const int base = i * 128 + q32 * 32;
+          const int lim = nkeys - base;
+          uint32_t m = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+          if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
+          return m;
+        };
+        // The row maximum over all 128 keys: this warp also reads the other
+        // half's S columns (only to take their maximum), so both warps of the
+        // row reach the same maximum and the same rescale decision without
+        // exchanging anything.
+        float mxp[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mxp[u] = -INFINITY;
+        {
+          float t[64];
+          tmem_ld32_async(tmem + lane_off + s * 128 + (half ^ 1) * 64, t);
+          tmem_ld32_async(tmem + lane_off + s * 128 + (half ^ 1) * 64 + 32, t + 32);
+          tmem_wait_ld_regs(t);
+          reg_fence32(t + 32);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t lv = live_bits((half ^ 1) * 2 + c);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              mxp[e & 3] = fmaxf(mxp[e & 3], ((lv >> e) & 1u) ? t[32 * c + e] : -INFINITY);
+          }
+        }
         float sv[64];
         tmem_ld32_async(tmem + lane_off + s * 128 + half * 64, sv);
         tmem_ld32_async(tmem + lane_off + s * 128 + half * 64 + 32, sv + 32);
@@ -379,35 +408,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&s_empty[s]);  // S now lives in registers: the buffer can take S of chunk g + 2
         // keys of this half that take part: bits of live[0] (keys 64h..64h+31) and live[1]
-        uint32_t live[2];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int base = i * 128 + half * 64 + c * 32;
-          const int lim = nkeys - base;
-          uint32_t m = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-          if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
-          live[c] = m;
-        }
+        const uint32_t live[2] = {live_bits(half * 2), live_bits(half * 2 + 1)};
         if ((live[0] & live[1]) != 0xffffffffu) {
 #pragma unroll
           for (int e = 0; e < 64; ++e)
             if (!((live[e >> 5] >> (e & 31)) & 1u)) sv[e] = -INFINITY;
         }
-        float mxp[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mxp[u] = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) mxp[e & 7] = fmaxf(mxp[e & 7], sv[e]);
-        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-        // combine with the other half of the row
-        float *xm = xmax + (s * 2) * 128;
-        xm[half * 128 + r] = mx;
-        if (!pair_sync()) {
-          ok = false;
-          break;
-        }
-        mx = fmaxf(mx, xm[(half ^ 1) * 128 + r]) * sl2;
+        for (int e = 0; e < 64; ++e) mxp[e & 3] = fmaxf(mxp[e & 3], sv[e]);
+        const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * sl2;
         const float m_new = fmaxf(m_used, mx);
         // lazy rescale: only when the max grows by more than 2^8 over the one in use
         const bool need = m_used != -INFINITY && m_new > m_used + kRescaleLog2;
@@ -467,25 +476,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       xs[half * 128 + r] = l;
       if (!pair_sync()) break;
       l += xs[(half ^ 1) * 128 + r];
-      // complement accumulator row, this half's 64 dimensions: the first 32 are
-      // loaded while P V of the last chunk runs, the rest (already pulled into
-      // L2 by the producers at the start of the tile) when they are merged.
-      // The compact cache holds them as bf16: acv[0..3] then carry the raw
-      // 16-byte words of the first 32.
+      // complement accumulator row, this half's 64 dimensions (pulled into L2
+      // by the producers at the start of the tile): the first kPre 16-byte
+      // words are loaded while P V of the last chunk runs, the rest when they
+      // are merged. The compact cache holds them as bf16 (8 words for all 64;
+      // acv then carries the raw words).
       const bool compact = p.compact != 0;
       const float4 *acg = compact ? nullptr : reinterpret_cast<const float4 *>(p.acc_c + row * 128 + half * 64);
       const uint4 *ocg = compact ? reinterpret_cast<const uint4 *>(p.o_c + row * 128 + half * 64) : nullptr;
-      float4 acv[8];
+      constexpr int kPre = 4;  // 16-byte words fetched early (more costs registers in the softmax loop)
+      float4 acv[kPre];
       if (MODE == kAttnDelta && gi < T) {
         if (compact) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < kPre; ++e) {
             const uint4 u = ocg[e];
             acv[e] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
           }
         } else {
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) acv[e4] = acg[e4];
+          for (int e4 = 0; e4 < kPre; ++e4) acv[e4] = acg[e4];
         }
       }
       if (nchunks > 0) {
@@ -526,9 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e8 = 0; e8 < 4; ++e8) {
               float av[8];  // complement accumulator (partial) or normalised output (compact), dims d0 + 8 e8 ..
               if (compact) {
-                const uint4 u = c == 0 ? make_uint4(__float_as_uint(acv[e8].x), __float_as_uint(acv[e8].y),
-                                                    __float_as_uint(acv[e8].z), __float_as_uint(acv[e8].w))
-                                       : ocg[4 + e8];
+                const int j = c * 4 + e8;
+                const uint4 u = j < kPre ? make_uint4(__float_as_uint(acv[j].x), __float_as_uint(acv[j].y),
+                                                      __float_as_uint(acv[j].z), __float_as_uint(acv[j].w))
+                                         : ocg[j];
                 const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -536,8 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   av[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
                 }
               } else {
-                const float4 a0 = c == 0 ? acv[2 * e8] : acg[8 + 2 * e8];
-                const float4 a1 = c == 0 ? acv[2 * e8 + 1] : acg[9 + 2 * e8];
+                const int j = c * 8 + 2 * e8;
+                const float4 a0 = j < kPre ? acv[j] : acg[j];
+                const float4 a1 = j + 1 < kPre ? acv[j + 1] : acg[j + 1];
                 av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w;
                 av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
               }

@@ -82,8 +82,9 @@ struct AttnParams {
   float *lse_c;
   uint16_t *o_c;
 };
-// tm_q: tile map over Q [T][h*128] (box 64 x 128). tm_k / tm_v: gather4 maps
-// (sparse step) or tile maps (dense, complement) over K, V [T][h*128].
+// tm_q: tile map over Q [T][h*128] (box 64 x 128). tm_k / tm_v: tile maps
+// over K, V [T][h*128] for the dense and complement passes (a sparse step
+// gathers the selected rows with cp.async and does not use them).
 cudaError_t launch_attn(int mode, const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                         const CUtensorMap &tm_v, cudaStream_t s);
 
