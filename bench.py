@@ -371,40 +371,62 @@ def run_gpu(args):
     status = cm.read_device_status()
     assert status == 0, f"device status {status}"
 
-    # end to end through the public API: pinned host inputs in, outputs back, every step
+    # End to end through the public API, every step's inputs copied in from pinned host memory
+    # and its outputs copied back, pipelined over three streams: step i + 1's inputs go up and
+    # step i - 1's outputs come down while step i computes (device inputs and outputs double
+    # buffered, events order the reuse; the caches update in place on the compute stream, step
+    # after step). The per-step working set (weights, caches, inputs: about 450 MB) is larger
+    # than L2, so the steps are not flushed in between. Per step = the whole run / steps.
     x_h = [x.cpu().pin_memory() for x in L.xs]
     qkv_h = [[t.cpu().pin_memory() for t in qkv] for qkv in L.qkvs]
     out_h = torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory()
     o_h = torch.empty(L.o.shape, dtype=L.o.dtype).pin_memory()
-    x_d = torch.empty_like(L.xs[0])
-    qkv_d = [torch.empty_like(t) for t in L.qkvs[0]]
+    x_d = [torch.empty_like(L.xs[0]) for _ in range(2)]
+    qkv_d = [[torch.empty_like(t) for t in L.qkvs[0]] for _ in range(2)]
+    out_d = [torch.empty_like(L.out) for _ in range(2)]
+    o_d = [torch.empty_like(L.o) for _ in range(2)]
+    s_cmp = torch.cuda.current_stream()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
     w_ = L.w
 
-    def e2e_step(i):
-        x_d.copy_(x_h[i % 2], non_blocking=True)
-        for dst, src in zip(qkv_d, qkv_h[i % 2]):
-            dst.copy_(src, non_blocking=True)
-        cm.mlp_delta(x_d, L.w1t, L.b1, L.w2, L.idx, L.a_cache, L.y_cache, L.out, Bt=w_["Bt"], workspace=L.ws)
-        cm.attn_delta(*qkv_d, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, scale=1 / math.sqrt(w_["d"]))
-        out_h.copy_(L.out, non_blocking=True)
-        o_h.copy_(L.o, non_blocking=True)
+    def e2e_run(nsteps):
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        ev_h, ev_c, ev_d = [ev() for _ in range(nsteps)], [ev() for _ in range(nsteps)], [ev() for _ in range(nsteps)]
+        start, end = ev(), ev()
+        start.record(s_h2d)
+        for i in range(nsteps):
+            b = i % 2
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(ev_c[i - 2])       # step i - 2 has read this input buffer
+                x_d[b].copy_(x_h[i % 2], non_blocking=True)
+                for dst, src in zip(qkv_d[b], qkv_h[i % 2]):
+                    dst.copy_(src, non_blocking=True)
+                ev_h[i].record(s_h2d)
+            s_cmp.wait_event(ev_h[i])
+            if i >= 2:
+                s_cmp.wait_event(ev_d[i - 2])           # step i - 2's outputs are downloaded
+            cm.mlp_delta(x_d[b], L.w1t, L.b1, L.w2, L.idx, L.a_cache, L.y_cache, out_d[b], Bt=w_["Bt"],
+                         workspace=L.ws, stream=s_cmp)
+            cm.attn_delta(*qkv_d[b], L.aidx, L.m_c, L.l_c, L.acc_c, o_d[b], scale=1 / math.sqrt(w_["d"]),
+                          stream=s_cmp)
+            ev_c[i].record(s_cmp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_c[i])
+                out_h.copy_(out_d[b], non_blocking=True)
+                o_h.copy_(o_d[b], non_blocking=True)
+                ev_d[i].record(s_d2h)
+        end.record(s_d2h)
+        end.synchronize()
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / nsteps
 
-    for i in range(min(args.warmup, 3)):
-        e2e_step(i)
+    e2e_run(max(args.warmup, 3))
     barrier()
     torch.cuda.synchronize()
-    e2e_ts = []
-    for i in range(args.steps):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        e2e_step(i)
-        b.record()
-        b.synchronize()
-        e2e_ts.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(e2e_run(args.steps), dev)
     barrier()
-    e2e_ms = max_over_ranks(statistics.mean(e2e_ts), dev)
-    h2d = x_d.numel() * 2 + sum(t.numel() * 2 for t in qkv_d)
+    h2d = x_d[0].numel() * 2 + sum(t.numel() * 2 for t in qkv_d[0])
     d2h = out_h.numel() * 2 + o_h.numel() * 2
 
     peaks, peak_src = load_peaks()
@@ -438,7 +460,8 @@ def run_gpu(args):
         "pct_bf16_peak": round(100 * flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 2),
         "kernels": kern, "roofline": roofline,
         "e2e": {"value": round(job_us_per_layer(e2e_ms, world), 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h),
+                "overlap": "step i+1 inputs up and step i-1 outputs down while step i computes (3 streams)"},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
