@@ -8,13 +8,13 @@
 // the selected key rows with 16-byte cp.async (one warp instruction = two
 // whole 256-byte key rows), on the dense passes one thread issues tiled TMA
 // loads. Warp 8 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
-// buffers, then O += P V into a TMEM accumulator (two, alternating between
-// tiles). Warps 0-7 run the online softmax, two warps per TMEM lane quadrant
-// (32 query rows), each on one 64-key half of S: both read the whole row to
-// take its maximum, exponentiate their half into P (bf16, a 128-byte-swizzled
-// shared tile, the A operand of the next P V) and rescale O in TMEM only when
-// the row maximum grows by more than 2^8. S of chunk i+1 is computed while
-// the softmax of chunk i runs. Logits are kept in log2 units (scale * log2 e).
+// buffers, then O += P V with P read from TMEM and V from shared memory.
+// Warps 0-7 run the online softmax, two warps per TMEM lane quadrant (32
+// query rows), each on one 64-key half of S: both read the whole row to take
+// its maximum, exponentiate their half into P (bf16 pairs stored into one of
+// two TMEM buffers with tcgen05.st) and rescale O in TMEM only when the row
+// maximum grows by more than 2^8. S of chunk i+1 is computed while the
+// softmax of chunk i runs. Logits are kept in log2 units (scale * log2 e).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -33,14 +33,13 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two 64-column swizzle halves)
 constexpr float kRescaleLog2 = 8.0f;     // O and l are rescaled only when the row max grows by more than 2^8
 
-// Shared memory: Q | K[2] | V[2] | P | barriers | key-index ring [4][128] |
+// Shared memory: Q | K[2] | V[2] | barriers | key-index ring [4][128] |
 // row-sum exchange [2][2][128] | key mask (complement pass).
 struct AttnCfg {
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kTileBytes;
   static constexpr uint32_t kVOff = kKOff + 2 * kTileBytes;
-  static constexpr uint32_t kPOff = kVOff + 2 * kTileBytes;
-  static constexpr uint32_t kBarOff = kPOff + kTileBytes;
+  static constexpr uint32_t kBarOff = kVOff + 2 * kTileBytes;
   static constexpr uint32_t kIdxOff = kBarOff + 256;
   static constexpr uint32_t kXsumOff = kIdxOff + 4 * 128 * 4;
   static constexpr uint32_t kMaskOff = kXsumOff + 2 * 2 * 128 * 4;
@@ -67,7 +66,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sQ = smem + C::kQOff;
   uint8_t *sK = smem + C::kKOff;
   uint8_t *sV = smem + C::kVOff;
-  uint8_t *sP = smem + C::kPOff;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
   uint64_t *q_full = bars + 0;
   uint64_t *q_empty = bars + 1;
@@ -77,10 +75,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *v_empty = bars + 8;    // [2] released when P V of the stage has been computed
   uint64_t *s_full = bars + 10;    // [2]
   uint64_t *s_empty = bars + 12;   // [2]
-  uint64_t *o_full = bars + 14;    // [2]
-  uint64_t *o_empty = bars + 16;   // [2]
-  uint64_t *p_full = bars + 18;
-  uint64_t *p_empty = bars + 19;
+  uint64_t *o_full = bars + 14;    // the last P V of the tile has landed in O
+  uint64_t *o_empty = bars + 15;   // the tile's epilogue has read O
+  uint64_t *p_full = bars + 16;    // [2] P of a chunk is in TMEM
+  uint64_t *p_empty = bars + 18;   // [2] P V of that chunk has been computed
   uint64_t *pair_bar = bars + 20;  // [4]: the two softmax warps of a lane quadrant exchange row partials
   uint64_t *kidx_bar = bars + 24;  // producers: a chunk's keys are staged
   uint64_t *mask_bar = bars + 25;  // softmax warps: complement mask steps
@@ -107,11 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], kSoftmaxThreads);
-      mbar_init(&o_full[s], 1);
-      mbar_init(&o_empty[s], kSoftmaxThreads);
+      mbar_init(&p_full[s], kSoftmaxThreads);
+      mbar_init(&p_empty[s], 1);
     }
-    mbar_init(p_full, kSoftmaxThreads);
-    mbar_init(p_empty, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, kSoftmaxThreads);
     for (int qd = 0; qd < 4; ++qd) mbar_init(&pair_bar[qd], 64);
     mbar_init(kidx_bar, kProducers);
     mbar_init(mask_bar, kSoftmaxThreads);
@@ -130,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S[0] at column 0, S[1] at 128, O[0] at 256, O[1] at 384
+  const uint32_t tmem = *tmem_slot;   // S[0] at column 0, S[1] at 128, O at 256, P[0] at 384, P[1] at 448
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ producers
@@ -257,12 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     int tl = 0;
     bool ok = true;
-    const uint32_t p0 = smem_u32(sP), q0 = smem_u32(sQ);
+    const uint32_t q0 = smem_u32(sQ);
+    const uint32_t tO = tmem + 256;
     for (int tile = blockIdx.x; tile < ntiles && ok && nchunks > 0; tile += gridDim.x, ++tl) {
-      const int ob = tl & 1;
-      const uint32_t tO = tmem + 256 + ob * 128;
       if (!wait_warp(q_full, tl & 1, p.status, abort_flag)) break;
-      if (!wait_warp(&o_empty[ob], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
       for (int i = 0; i <= nchunks && ok; ++i) {
         if (i < nchunks) {
           const int g = tl * nchunks + i, s = g & 1;
@@ -288,23 +284,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
         if (i >= 1) {
+          // P V: A = P from TMEM (buffer g & 1), B = V from shared memory
           const int j = i - 1, g = tl * nchunks + j, s = g & 1;
-          if (!wait_warp(p_full, g & 1, p.status, abort_flag) ||
+          // O is free once the previous tile's epilogue has read it (S of this tile went ahead)
+          if (j == 0 && !wait_warp(o_empty, (tl & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (!wait_warp(&p_full[s], (g >> 1) & 1, p.status, abort_flag) ||
               !wait_warp(&v_full[s], (g >> 1) & 1, p.status, abort_flag)) {
             ok = false;
             break;
           }
-          fence_async_smem();
+          if (MODE == kAttnDelta) fence_async_smem();
           tc_fence_after();
           if (lane == 0) {
             const uint32_t v0 = smem_u32(sV + s * kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_bf16(tO, sdesc_sw128(p0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                        sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV, (j | kk) != 0);
+              umma_bf16_ts(tO, tmem + 384 + s * 64 + kk * 8, sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV,
+                           (j | kk) != 0);
             umma_commit(&v_empty[s]);
-            umma_commit(p_empty);
-            if (j == nchunks - 1) umma_commit(&o_full[ob]);
+            umma_commit(&p_empty[s]);
+            if (j == nchunks - 1) umma_commit(o_full);
           }
           __syncwarp();
         }
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hh = tile % p.h, b = tile / p.h;
       const int gi = b * 128 + r;
       const int ob = tl & 1;
-      const uint32_t tO = tmem + lane_off + 256 + ob * 128 + half * 64;
+      const uint32_t tO = tmem + lane_off + 256 + half * 64;
       if (MODE == kAttnComplement) {
         // mask of the keys this tile's block selected
         const int nwords = (T + 31) >> 5;
@@ -422,8 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need = m_used != -INFINITY && m_new > m_used + kRescaleLog2;
         if (m_used == -INFINITY) m_used = m_new;
         if (__any_sync(0xffffffffu, need)) {
-          // O holds P V of the earlier chunks: wait for the last of them, then scale this half in TMEM
-          if (!wait_warp(p_empty, (g & 1) ^ 1, p.status, abort_flag)) {
+          // O holds P V of the earlier chunks (i >= 1 here): wait for the last of them, then
+          // scale this half in TMEM
+          if (!wait_warp(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, p.status, abort_flag)) {
             ok = false;
             break;
           }
@@ -453,22 +456,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           lp[e & 3] += sv[e];
         }
         l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-        // P of the previous chunk must have been consumed before it is overwritten
-        if (!wait_warp(p_empty, (g & 1) ^ 1, p.status, abort_flag)) {
+        // P into TMEM buffer g & 1 (this row's keys 64h .. 64h+63 as 32 columns of
+        // bf16 pairs), once P V of chunk g - 2 has read that buffer
+        if (!wait_warp(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t *prow = sP + half * 16384 + r * 128;
+        uint32_t pk[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {  // 16-byte chunk c8 = keys 64h + 8*c8 .. +7
-          const float *pv = sv + 8 * c8;
-          *reinterpret_cast<uint4 *>(prow + ((c8 ^ (r & 7)) << 4)) =
-              make_uint4(cvt_bf16x2(pv[0], pv[1]), cvt_bf16x2(pv[2], pv[3]), cvt_bf16x2(pv[4], pv[5]),
-                         cvt_bf16x2(pv[6], pv[7]));
-        }
-        fence_async_smem();
-        tc_fence_before();  // orders a rescale's TMEM stores before the next P V
-        mbar_arrive(p_full);
+        for (int e = 0; e < 32; ++e) pk[e] = cvt_bf16x2(sv[2 * e], sv[2 * e + 1]);
+        tmem_st32(tmem + lane_off + 384 + (g & 1) * 64 + half * 32, reinterpret_cast<const float *>(pk));
+        tmem_wait_st();
+        tc_fence_before();  // orders the P stores (and a rescale's O stores) before the next P V
+        mbar_arrive(&p_full[g & 1]);
       }
       if (!ok) break;
       // row sum over both halves (buffer by tile parity: the next write to it is two tiles away)
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (nchunks > 0) {
-        if (!wait_warp(&o_full[ob], (tl >> 1) & 1, p.status, abort_flag)) break;
+        if (!wait_warp(o_full, tl & 1, p.status, abort_flag)) break;
         tc_fence_after();
       }
       const float m2 = m_used;
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tO + c * 32, ov);
           if (c == 1) {
             tc_fence_before();
-            mbar_arrive(&o_empty[ob]);
+            mbar_arrive(o_empty);
           }
         } else {
 #pragma unroll
