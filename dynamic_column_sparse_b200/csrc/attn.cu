@@ -51,8 +51,10 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *s
 }
 
 
-// Persistent: each CTA walks tiles (head, 128-query block) blockIdx.x,
-// blockIdx.x + gridDim.x, ...; every tile has the same number of key chunks,
+// Persistent: each CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...,
+// tile t = head * nb + query block (head-major, so the CTAs running at the
+// same time gather from one head's keys and values, which stay in L2 even
+// when all heads' do not); every tile has the same number of key chunks,
 // so all roles index chunks by one running counter g.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // selected keys of chunk g, rows pt and pt + 96 (the latter for pt < 32)
     auto load_keys = [&](int g, int &ka, int &kb2) {
       const int tile = blockIdx.x + (g / nchunks) * gridDim.x, i = g % nchunks;
-      const int hh = tile % p.h, b = tile / p.h;
+      const int hh = tile / p.nb, b = tile % p.nb;
       const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
       ka = __ldg(irow + min(i * 128 + pt, p.k - 1));
       kb2 = pt < 32 ? __ldg(irow + min(i * 128 + pt + 96, p.k - 1)) : 0;
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g0 = 0;
     for (int tl = 0; tl < my_tiles && ok && nchunks > 0; ++tl, g0 += nchunks) {
       const int tile = blockIdx.x + tl * gridDim.x;
-      const int hh = tile % p.h, b = tile / p.h;
+      const int hh = tile / p.nb, b = tile % p.nb;
       if (pw == 0) {
         if (!wait_warp(q_empty, (tl & 1) ^ 1, p.status, abort_flag)) break;
         if (lane == 0) {
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tl = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
-      const int hh = tile % p.h, b = tile / p.h;
+      const int hh = tile / p.nb, b = tile % p.nb;
       const int gi = b * 128 + r;
       const int ob = tl & 1;
       const uint32_t tO = tmem + lane_off + 256 + half * 64;
@@ -631,8 +633,9 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
-  const int hh = blockIdx.x % p.h;
-  const int b = blockIdx.x / p.h;
+  // head-major: blocks that run at the same time read the same head's keys (L2 reuse)
+  const int hh = blockIdx.x / p.nb;
+  const int b = blockIdx.x % p.nb;
   const int T = p.T;
   const int nchunks = (T + 127) / 128;
 
