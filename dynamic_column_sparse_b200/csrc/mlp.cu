@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
 }
 
 template <int BN>
-struct DownCfg : Roles<4, 4> {
+struct DownCfg : Roles<8, 4> {   // eight gathering warps: the W2 stream is bound by cp.async issue per warp
   static constexpr int kCtasPerSm = 1;
   static constexpr int kAccs = 2;                        // TMEM accumulators (kAccs * BN columns)
   static constexpr int kStagesA = 3;                     // delta tile
