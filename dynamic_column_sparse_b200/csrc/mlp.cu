@@ -17,7 +17,8 @@
 // warps with cp.async (one warp instruction = whole row segments); both
 // operands are MN-major. The epilogue adds the fp32 result into the output
 // cache (or overwrites it with result + b2 on a refresh) and writes the bf16
-// layer output.
+// layer output; each warp turns its 32 x 32 accumulator chunks around in
+// shared memory first, so those accesses are whole-line runs.
 //
 // Each kernel keeps two shared-memory rings: one for the gathered operand
 // (filled by the cp.async producer warps) and one for the operand that
@@ -367,7 +368,8 @@ struct DownCfg : Roles<8, 4> {   // eight gathering warps: the W2 stream is boun
   static constexpr uint32_t kBBytes = (BN / 64) * 8192;  // 64 K-rows x BN columns
   static constexpr uint32_t kBOff = kStagesA * kABytes;
   static constexpr uint32_t kBarOff = kBOff + kStagesB * kBBytes;
-  static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
+  static constexpr uint32_t kEpiOff = kBarOff + 1024;   // per epilogue warp: 32 x 33 fp32 transpose buffer
+  static constexpr uint32_t kSmem = 1024 + kEpiOff + kEpiWarps * 32 * 33 * 4;
 };
 
 // Persistent: CTA c handles tiles c, c + gridDim.x, ...; the two TMEM
@@ -578,14 +580,21 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
       __syncwarp();
     }
   } else {
+    // epilogue: warp w reads TMEM lane quadrant q = w % 4 (tokens 32q ..
+    // 32q + 31, one per thread) 32 columns at a time and turns the chunk
+    // around in its shared buffer (rows padded to 33 words, so both the
+    // row-wise writes and the column-wise reads are free of bank conflicts);
+    // then eight lanes cover one token's 32 columns, and every access to the
+    // output cache and the layer output is a whole 128-byte (64-byte) run.
+    static_assert(C::kEpiWarps == 4, "one epilogue warp per TMEM lane quadrant");
     const int q = warp & 3;
-    const int t = q * 32 + lane;
+    float *ebuf = reinterpret_cast<float *>(smem + C::kEpiOff) + (warp - C::kEpiWarp0) * (32 * 33);
+    const int rsub = lane >> 3, c4 = (lane & 7) * 4;   // row within a group of four, first column
+    const bool accumulate = p.mode == kDownAccumulate;
     int tl = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
       const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
       const int ab = tl % C::kAccs;
-      const int64_t grow = static_cast<int64_t>(b) * BT + t;
-      const bool valid = t < BT && grow < p.T;
       if (!wait_warp(&acc_full[ab], (tl / C::kAccs) & 1, p.status, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -596,33 +605,37 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
         }
-        if (valid) {
-          const int n = n0 + nc * 32;
-          float4 *y4 = reinterpret_cast<float4 *>(p.y_cache + grow * p.D + n);
-          float y[32];
-          if (p.mode == kDownAccumulate) {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float4 o = y4[v];
-              y[4 * v] = o.x + acc[4 * v];
-              y[4 * v + 1] = o.y + acc[4 * v + 1];
-              y[4 * v + 2] = o.z + acc[4 * v + 2];
-              y[4 * v + 3] = o.w + acc[4 * v + 3];
-            }
-          } else {
+        for (int i = 0; i < 32; ++i) ebuf[lane * 33 + i] = acc[i];
+        __syncwarp();
+        const int n = n0 + nc * 32 + c4;
+        float4 old[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) y[i] = acc[i] + bf16_bits_to_f32(__ldg(p.b2 + n + i));
-          }
+        for (int g = 0; g < 8; ++g) {
+          const int r = q * 32 + 4 * g + rsub;               // token within the block
+          const int64_t grow = static_cast<int64_t>(b) * BT + r;
+          if (accumulate && r < BT && grow < p.T)
+            old[g] = *reinterpret_cast<const float4 *>(p.y_cache + grow * p.D + n);
+        }
+        float4 bias = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!accumulate)
+          bias = make_float4(bf16_bits_to_f32(__ldg(p.b2 + n)), bf16_bits_to_f32(__ldg(p.b2 + n + 1)),
+                             bf16_bits_to_f32(__ldg(p.b2 + n + 2)), bf16_bits_to_f32(__ldg(p.b2 + n + 3)));
 #pragma unroll
-          for (int v = 0; v < 8; ++v) y4[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
-          if (p.out != nullptr) {
-            uint4 *o4 = reinterpret_cast<uint4 *>(p.out + grow * p.D + n);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              o4[v] = make_uint4(cvt_bf16x2(y[8 * v], y[8 * v + 1]), cvt_bf16x2(y[8 * v + 2], y[8 * v + 3]),
-                                 cvt_bf16x2(y[8 * v + 4], y[8 * v + 5]), cvt_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+        for (int g = 0; g < 8; ++g) {
+          const int rr = 4 * g + rsub;                       // row of the warp's quadrant
+          const int r = q * 32 + rr;
+          const int64_t grow = static_cast<int64_t>(b) * BT + r;
+          if (r < BT && grow < p.T) {
+            const float *e = ebuf + rr * 33 + c4;
+            const float4 base = accumulate ? old[g] : bias;
+            const float4 y = make_float4(base.x + e[0], base.y + e[1], base.z + e[2], base.w + e[3]);
+            *reinterpret_cast<float4 *>(p.y_cache + grow * p.D + n) = y;
+            if (p.out != nullptr)
+              *reinterpret_cast<uint2 *>(p.out + grow * p.D + n) = make_uint2(cvt_bf16x2(y.x, y.y), cvt_bf16x2(y.z, y.w));
           }
         }
+        __syncwarp();  // the buffer is rewritten by the next chunk
       }
     }
   }
