@@ -8,8 +8,9 @@
 // brings them instead. The token block of x arrives by a tiled TMA load. One
 // thread issues tcgen05 bf16 MMAs accumulating D[col][token] in one of two
 // TMEM accumulators. Each epilogue thread owns one hidden column (one TMEM
-// lane) and half of the block's tokens, so the activation cache run
-// a_cache[b][c][..] and the delta row are read and written as contiguous runs.
+// lane); the activation cache runs a_cache[b][c][..] and the delta rows are
+// moved 64 bytes per run between global memory and a per-warp shared buffer
+// that turns them around to and from that layout.
 //
 // Kernel 2 (mlp_down): one CTA per (token block b, slice of BN model columns).
 // K runs over the selected hidden units: the delta rows come from the
@@ -64,7 +65,9 @@ struct UpCfg : Roles<4, 4> {
   static constexpr uint32_t kBOff = kStagesA * kABytes;
   static constexpr uint32_t kPartOff = kBOff + kStagesB * kBBytes;  // [2][128] fp32 partial column scores
   static constexpr uint32_t kBarOff = kPartOff + 2 * 128 * 4;
-  static constexpr uint32_t kSmem = 1024 + kBarOff + 1024;
+  static constexpr uint32_t kTbBytes = 32 * 80;  // per epilogue warp: 32 columns x 32 tokens bf16, rows padded to 80 B
+  static constexpr uint32_t kEpiOff = kBarOff + 1024;
+  static constexpr uint32_t kSmem = 1024 + kEpiOff + kEpiWarps * kTbBytes;
 };
 
 // Persistent: CTA c handles tiles c, c + gridDim.x, ... where tile = chunk * nb
@@ -254,13 +257,20 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       __syncwarp();
     }
   } else {
-    // epilogue: thread = one selected column (TMEM lane r) and 1 / kParts of the block's tokens
+    // epilogue: thread = one selected column (TMEM lane r) and 1 / kParts of
+    // the block's tokens, 32 tokens at a time. The cached activations and the
+    // delta rows are moved between global memory and the warp's shared buffer
+    // as whole 64-byte runs (lane: 16-byte piece lane % 4 of the columns
+    // 8 i + lane / 4), and turned around there to and from the one-column-per-
+    // thread layout of the accumulator.
     const int ew = warp - C::kEpiWarp0;
     const int q = warp & 3;
     const int th = ew >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const bool first = p.mode == kUpRefreshFirst;
+    uint8_t *tb = smem + C::kEpiOff + ew * C::kTbBytes;
+    const int ck = lane & 3, cq = lane >> 2;
     for (int tl = 0; tl < my_tiles; ++tl) {
       const int tile = blockIdx.x + tl * gridDim.x;
       const int chunk = tile / p.nb, b = tile % p.nb;
@@ -280,65 +290,100 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       }
       const float bias = bf16_bits_to_f32(__ldg(p.b1 + c));
       const int nvalid = min(BT, p.T - b * BT);
-      uint16_t *arow = p.a_cache + (static_cast<size_t>(b) * p.H + c) * BT + th * kHalf;
-      uint16_t *drow = sparse ? p.delta + (static_cast<size_t>(b) * p.k_pad + j) * BT + th * kHalf : nullptr;
-      // the first 32 of this warp's tokens are fetched here, the rest in the loop below
-      constexpr int kPre = 1;
       const bool need_old = valid_j && !(first && !sparse);
-      uint4 oldv[kPre * 4];
+      // the columns whose runs this lane moves: 8 i + cq, i = 0..3
+      int ci_of[4];
+      uint32_t val_mask = 0, old_mask = 0;
 #pragma unroll
-      for (int v = 0; v < kPre * 4; ++v)
-        oldv[v] = need_old ? reinterpret_cast<const uint4 *>(arow)[v] : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) {
+        ci_of[i] = __shfl_sync(0xffffffffu, c, 8 * i + cq);
+        val_mask |= __shfl_sync(0xffffffffu, valid_j ? 1u : 0u, 8 * i + cq) << i;
+        old_mask |= __shfl_sync(0xffffffffu, need_old ? 1u : 0u, 8 * i + cq) << i;
+      }
+      const size_t a_off = static_cast<size_t>(b) * p.H * BT + th * kHalf + ck * 8;
+      auto arun = [&](int i) { return p.a_cache + a_off + static_cast<size_t>(ci_of[i]) * BT; };
+      uint16_t *drun0 = sparse ? p.delta + (static_cast<size_t>(b) * p.k_pad + chunk * 128 + q * 32 + cq) * BT +
+                                     th * kHalf + ck * 8
+                               : nullptr;
+      uint4 pre[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        pre[i] = (old_mask >> i) & 1 ? *reinterpret_cast<const uint4 *>(arun(i)) : make_uint4(0, 0, 0, 0);
       if (!wait_warp(&acc_full[ab], (tl >> 1) & 1, p.status, abort_flag)) break;
       tc_fence_after();
       float score = 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int tq = 0; tq < kHalf / 32; ++tq) {
+        // old activations of tokens 32 tq .. into the buffer, then this thread's column out of it
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4 *>(tb + (8 * i + cq) * 80 + ck * 16) = pre[i];
+        __syncwarp();
+        uint4 oldw[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) oldw[v] = *reinterpret_cast<const uint4 *>(tb + lane * 80 + v * 16);
         float acc[32];
         tmem_ld32(tmem + lane_off + ab * BT + th * kHalf + tq * 32, acc);
         if (tq == kHalf / 32 - 1) {
           tc_fence_before();
           mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
         }
-        uint4 oldl[4];
-        if (tq >= kPre) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            oldl[v] = need_old ? reinterpret_cast<const uint4 *>(arow + tq * 32)[v] : make_uint4(0, 0, 0, 0);
-        }
-        const uint16_t *old = reinterpret_cast<const uint16_t *>(tq < kPre ? oldv + tq * 4 : oldl);
-        uint32_t na[16], dl[16];
+        const uint16_t *old = reinterpret_cast<const uint16_t *>(oldw);
+        uint32_t na[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          uint16_t nab[2], dlb[2];
+          uint16_t nab[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = th * kHalf + tq * 32 + i + u;
             const float a = gelu_tanh(acc[i + u] + bias);
-            const uint16_t abf = f32_to_bf16_bits(a);
             const bool tok = t < nvalid;
-            const float o = bf16_bits_to_f32(old[i + u]);
-            nab[u] = tok ? abf : old[i + u];
-            if (sparse) {
-              dlb[u] = (valid_j && tok) ? f32_to_bf16_bits(bf16_bits_to_f32(abf) - o) : static_cast<uint16_t>(0);
-            } else {
-              dlb[u] = 0;
-              score += tok ? fabsf(first ? a : a - o) : 0.f;
-            }
+            nab[u] = tok ? f32_to_bf16_bits(a) : old[i + u];
+            if (!sparse) score += tok ? fabsf(first ? a : a - bf16_bits_to_f32(old[i + u])) : 0.f;
           }
           na[i / 2] = static_cast<uint32_t>(nab[0]) | (static_cast<uint32_t>(nab[1]) << 16);
-          dl[i / 2] = static_cast<uint32_t>(dlb[0]) | (static_cast<uint32_t>(dlb[1]) << 16);
         }
-        if (valid_j) {
-          uint4 *dst = reinterpret_cast<uint4 *>(arow + tq * 32);
+        // new activations back through the buffer as whole runs
+        __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(na[4 * v], na[4 * v + 1], na[4 * v + 2], na[4 * v + 3]);
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4 *>(tb + lane * 80 + v * 16) = make_uint4(na[4 * v], na[4 * v + 1], na[4 * v + 2], na[4 * v + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if ((val_mask >> i) & 1)
+            *reinterpret_cast<uint4 *>(arun(i) + tq * 32) = *reinterpret_cast<const uint4 *>(tb + (8 * i + cq) * 80 + ck * 16);
+        // the next chunk's old activations are in flight while the delta goes out
+        if (tq + 1 < kHalf / 32) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            pre[i] = (old_mask >> i) & 1 ? *reinterpret_cast<const uint4 *>(arun(i) + (tq + 1) * 32) : make_uint4(0, 0, 0, 0);
         }
         if (sparse) {
-          uint4 *dst = reinterpret_cast<uint4 *>(drow + tq * 32);
+          // delta = bf16(new) - old for real tokens of a selected column, else 0
+          const uint16_t *nw = reinterpret_cast<const uint16_t *>(na);
+          uint32_t dl[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(dl[4 * v], dl[4 * v + 1], dl[4 * v + 2], dl[4 * v + 3]);
+          for (int i = 0; i < 32; i += 2) {
+            uint16_t dlb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const bool tok = th * kHalf + tq * 32 + i + u < nvalid;
+              dlb[u] = (valid_j && tok) ? f32_to_bf16_bits(bf16_bits_to_f32(nw[i + u]) - bf16_bits_to_f32(old[i + u]))
+                                        : static_cast<uint16_t>(0);
+            }
+            dl[i / 2] = static_cast<uint32_t>(dlb[0]) | (static_cast<uint32_t>(dlb[1]) << 16);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4 *>(tb + lane * 80 + v * 16) = make_uint4(dl[4 * v], dl[4 * v + 1], dl[4 * v + 2], dl[4 * v + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4 *>(drun0 + static_cast<size_t>(8 * i) * BT + tq * 32) =
+                *reinterpret_cast<const uint4 *>(tb + (8 * i + cq) * 80 + ck * 16);
         }
+        __syncwarp();  // the buffer takes the next chunk's old activations
       }
       if (!sparse && kParts == 1) {
         if (valid_j) p.scores[static_cast<size_t>(b) * p.H + c] = score;
