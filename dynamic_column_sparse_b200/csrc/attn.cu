@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [4][128] selected keys of chunk g at g & 3
   float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
   uint32_t *mask = reinterpret_cast<uint32_t *>(smem + C::kMaskOff);
+  float *ebuf = reinterpret_cast<float *>(smem + C::kMaskOff);      // delta pass: [8 warps][32][36] merge buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
@@ -478,28 +479,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       xs[half * 128 + r] = l;
       if (!pair_sync()) break;
       l += xs[(half ^ 1) * 128 + r];
-      // complement accumulator row, this half's 64 dimensions (pulled into L2
-      // by the producers at the start of the tile): the first kPre 16-byte
-      // words are loaded while P V of the last chunk runs, the rest when they
-      // are merged. The compact cache holds them as bf16 (8 words for all 64;
-      // acv then carries the raw words).
+      // Delta pass: the complement rows of this warp's 32 queries (this half's
+      // 64 dimensions, pulled into L2 by the producers at the start of the
+      // tile) and the output rows move as whole runs through the warp's shared
+      // buffer (rows padded to 36 words): fp32 lane = query 4 i + lane / 8,
+      // 16-byte piece lane % 8 of a 32-dimension group; bf16 (the compact
+      // cache, the output) lane = query 8 i + lane / 4, piece lane % 4. The
+      // first group is loaded while P V of the last chunk runs, the second
+      // while the first is merged.
       const bool compact = p.compact != 0;
-      const float4 *acg = compact ? nullptr : reinterpret_cast<const float4 *>(p.acc_c + row * 128 + half * 64);
-      const uint4 *ocg = compact ? reinterpret_cast<const uint4 *>(p.o_c + row * 128 + half * 64) : nullptr;
-      constexpr int kPre = 4;  // 16-byte words fetched early (more costs registers in the softmax loop)
-      float4 acv[kPre];
-      if (MODE == kAttnDelta && gi < T) {
-        if (compact) {
+      float *eb = ebuf + warp * (32 * 36);
+      const int qbase = b * 128 + q * 32;
+      float4 gv[8];
+      auto load_group = [&](int c) {
+        const int d = half * 64 + c * 32;
+        if (!compact) {
 #pragma unroll
-          for (int e = 0; e < kPre; ++e) {
-            const uint4 u = ocg[e];
-            acv[e] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+          for (int i = 0; i < 8; ++i) {
+            const int gq = qbase + 4 * i + (lane >> 3);
+            gv[i] = gq < T ? *reinterpret_cast<const float4 *>(p.acc_c + (static_cast<size_t>(hh) * T + gq) * 128 + d +
+                                                               4 * (lane & 7))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         } else {
 #pragma unroll
-          for (int e4 = 0; e4 < kPre; ++e4) acv[e4] = acg[e4];
+          for (int i = 0; i < 4; ++i) {
+            const int gq = qbase + 8 * i + (lane >> 2);
+            const uint4 u = gq < T ? *reinterpret_cast<const uint4 *>(p.o_c + (static_cast<size_t>(hh) * T + gq) * 128 +
+                                                                      d + 8 * (lane & 3))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            gv[i] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+          }
         }
-      }
+      };
+      if (MODE == kAttnDelta) load_group(0);
       if (nchunks > 0) {
         if (!wait_warp(o_full, tl & 1, p.status, abort_flag)) break;
         tc_fence_after();
@@ -530,38 +543,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0.f;
         }
-        if (gi < T) {
-          const int d0 = half * 64 + c * 32;
-          if (MODE == kAttnDelta) {
-            uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
+        const int d0 = half * 64 + c * 32;
+        if (MODE == kAttnDelta) {
+          // the group's complement values into the buffer, then this thread's row out of it
+          if (!compact) {
 #pragma unroll
-            for (int e8 = 0; e8 < 4; ++e8) {
-              float av[8];  // complement accumulator (partial) or normalised output (compact), dims d0 + 8 e8 ..
-              if (compact) {
-                const int j = c * 4 + e8;
-                const uint4 u = j < kPre ? make_uint4(__float_as_uint(acv[j].x), __float_as_uint(acv[j].y),
-                                                      __float_as_uint(acv[j].z), __float_as_uint(acv[j].w))
-                                         : ocg[j];
-                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4 *>(eb + (4 * i + (lane >> 3)) * 36 + 4 * (lane & 7)) = gv[i];
+          } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  av[2 * j] = __uint_as_float(w4[j] << 16);
-                  av[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
-                }
-              } else {
-                const int j = c * 8 + 2 * e8;
-                const float4 a0 = j < kPre ? acv[j] : acg[j];
-                const float4 a1 = j + 1 < kPre ? acv[j + 1] : acg[j + 1];
-                av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w;
-                av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<float4 *>(eb + (8 * i + (lane >> 2)) * 36 + 4 * (lane & 3)) = gv[i];
+          }
+          __syncwarp();
+          if (c == 0) load_group(1);
+          uint32_t w[16];
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            float av[8];  // complement accumulator (partial) or normalised output (compact), dims d0 + 8 e8 ..
+            if (compact) {
+              const uint4 u = *reinterpret_cast<const uint4 *>(eb + lane * 36 + 4 * e8);
+              const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                av[2 * j] = __uint_as_float(w4[j] << 16);
+                av[2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
               }
-              const float *oa = ov + 8 * e8;
-              orow[e8] = make_uint4(cvt_bf16x2((av[0] * wc + oa[0] * ws) * inv, (av[1] * wc + oa[1] * ws) * inv),
-                                    cvt_bf16x2((av[2] * wc + oa[2] * ws) * inv, (av[3] * wc + oa[3] * ws) * inv),
-                                    cvt_bf16x2((av[4] * wc + oa[4] * ws) * inv, (av[5] * wc + oa[5] * ws) * inv),
-                                    cvt_bf16x2((av[6] * wc + oa[6] * ws) * inv, (av[7] * wc + oa[7] * ws) * inv));
+            } else {
+              const float4 a0 = *reinterpret_cast<const float4 *>(eb + lane * 36 + 8 * e8);
+              const float4 a1 = *reinterpret_cast<const float4 *>(eb + lane * 36 + 8 * e8 + 4);
+              av[0] = a0.x, av[1] = a0.y, av[2] = a0.z, av[3] = a0.w;
+              av[4] = a1.x, av[5] = a1.y, av[6] = a1.z, av[7] = a1.w;
             }
-          } else if (MODE == kAttnDense) {
+            const float *oa = ov + 8 * e8;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              w[4 * e8 + j] = cvt_bf16x2((av[2 * j] * wc + oa[2 * j] * ws) * inv, (av[2 * j + 1] * wc + oa[2 * j + 1] * ws) * inv);
+          }
+          // the merged row (bf16) back into the buffer, then out as whole runs
+          __syncwarp();
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4 *>(eb + lane * 36 + 4 * v) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = 8 * i + (lane >> 2);
+            const int gq = qbase + rr;
+            if (gq < T)
+              *reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gq) * p.h + hh) * 128 + d0 + 8 * (lane & 3)) =
+                  *reinterpret_cast<const uint4 *>(eb + rr * 36 + 4 * (lane & 3));
+          }
+          __syncwarp();  // the buffer takes the next group
+        } else if (gi < T) {
+          if (MODE == kAttnDense) {
             uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(gi) * p.h + hh) * 128 + d0);
 #pragma unroll
             for (int e8 = 0; e8 < 4; ++e8) {
@@ -733,7 +768,8 @@ __global__ void __launch_bounds__(kMassThreads, 1)
 template <int MODE>
 uint32_t attn_smem(int64_t T) {
   const uint32_t mask_bytes = MODE == kAttnComplement ? ((static_cast<uint32_t>(T) + 31) / 32) * 4 : 0;
-  return 1024 + AttnCfg::kMaskOff + mask_bytes;
+  const uint32_t merge_bytes = MODE == kAttnDelta ? 8 * 32 * 36 * 4 : 0;
+  return 1024 + AttnCfg::kMaskOff + mask_bytes + merge_bytes;
 }
 
 template <int MODE>
