@@ -4,7 +4,7 @@
 //
 // Persistent CTAs walk (head, 128-query block) tiles. Q arrives once per tile
 // by a tiled TMA load; K and V stream in chunks of 128 keys through two-stage
-// rings, K one chunk ahead of V: on a sparse step producer warps 9-11 gather
+// rings, K one chunk ahead of V: on a sparse step producer warps 9-15 gather
 // the selected key rows with 16-byte cp.async (one warp instruction = two
 // whole 256-byte key rows), on the dense passes one thread issues tiled TMA
 // loads. Warp 8 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
@@ -23,11 +23,11 @@
 namespace cm {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kSoftmaxThreads = 256;   // warps 0-7: two warps per TMEM lane quadrant, one per half of the columns
 constexpr int kMmaWarp = 8;
-constexpr int kProdWarp0 = 9;          // warps 9-11
-constexpr int kProducers = 96;
+constexpr int kProdWarp0 = 9;          // warps 9-15
+constexpr int kProducers = 224;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two 64-column swizzle halves)
@@ -82,7 +82,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *p_full = bars + 16;    // [2] P of a chunk is in TMEM
   uint64_t *p_empty = bars + 18;   // [2] P V of that chunk has been computed
   uint64_t *pair_bar = bars + 20;  // [4]: the two softmax warps of a lane quadrant exchange row partials
-  uint64_t *kidx_bar = bars + 24;  // producers: a chunk's keys are staged
   uint64_t *mask_bar = bars + 25;  // softmax warps: complement mask steps
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -114,7 +113,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_full, 1);
     mbar_init(o_empty, kSoftmaxThreads);
     for (int qd = 0; qd < 4; ++qd) mbar_init(&pair_bar[qd], 64);
-    mbar_init(kidx_bar, kProducers);
     mbar_init(mask_bar, kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
@@ -141,23 +139,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ahead of V; the last V of a tile goes out before the next tile's loads.
     // g counts chunks over this CTA's tiles.
     const int pw = warp - kProdWarp0;
-    const int pt = threadIdx.x - kProdWarp0 * 32;  // 0..95
+    const int pt = threadIdx.x - kProdWarp0 * 32;  // 0..223
     const int my_tiles = static_cast<int>(blockIdx.x) < ntiles ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
     const int total = my_tiles * nchunks;
-    // selected keys of chunk g, rows pt and pt + 96 (the latter for pt < 32)
-    auto load_keys = [&](int g, int &ka, int &kb2) {
+    // warp pw moves rows 20 pw .. 20 pw + 19 (< 128) of every chunk and
+    // stages their selected keys itself (lane l: row 20 pw + l), so the
+    // producer warps never wait for one another
+    constexpr int kRowsPerWarp = 20;
+    const int krow = pw * kRowsPerWarp + lane;
+    const bool kload = lane < kRowsPerWarp && krow < 128;
+    auto load_keys = [&](int g, int &ka) {
       const int tile = blockIdx.x + (g / nchunks) * gridDim.x, i = g % nchunks;
       const int hh = tile / p.nb, b = tile % p.nb;
       const int32_t *irow = p.idx + (static_cast<size_t>(hh) * p.nb + b) * p.k;
-      ka = __ldg(irow + min(i * 128 + pt, p.k - 1));
-      kb2 = pt < 32 ? __ldg(irow + min(i * 128 + pt + 96, p.k - 1)) : 0;
+      ka = kload ? __ldg(irow + min(i * 128 + krow, p.k - 1)) : 0;
     };
-    // warp pw moves the row pairs (2q, 2q+1), q = 22 pw .. 22 pw + 21 (< 64):
-    // lanes 0-15 the even row, 16-31 the odd one, 16 bytes each. The warp's
-    // keys are read from shared memory up front, so the copies issue back to
-    // back with one address computation each.
+    // the row pairs (2q, 2q+1), q = 10 pw .. 10 pw + 9 (< 64): lanes 0-15 the
+    // even row, 16-31 the odd one, 16 bytes each. The keys are read from
+    // shared memory up front, so the copies issue back to back with one
+    // address computation each.
     auto gather = [&](const uint16_t *src, uint8_t *dst, const int *ks, int hh) {
-      constexpr int kPairs = 22;
+      constexpr int kPairs = kRowsPerWarp / 2;
       const int c16 = lane & 15, hi = lane >> 4;
       const uint16_t *lb = src + hh * 128 + c16 * 8;
       const size_t rs = static_cast<size_t>(p.h) * 128;
@@ -174,9 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    int ka = 0, kb2 = 0;
-    if (MODE == kAttnDelta && total > 0) load_keys(0, ka, kb2);
-    uint32_t kidx_phase = 0;
+    int ka = 0;
+    if (MODE == kAttnDelta && total > 0) load_keys(0, ka);
     // K of chunk g (i = its index in the tile), for the tile's head / block
     auto load_k = [&](int g, int i, int hh) -> bool {
       const int s = g & 1;
@@ -184,18 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (MODE == kAttnDelta) {
         // stage the chunk's keys in slot g & 3 (read again for V two loads
         // later), range-checked, then fetch the next chunk's while the copies go out
-        if (static_cast<unsigned>(ka) >= static_cast<unsigned>(T) || static_cast<unsigned>(kb2) >= static_cast<unsigned>(T)) {
+        if (static_cast<unsigned>(ka) >= static_cast<unsigned>(T)) {
           atomicCAS(p.status, kDevOk, kDevBadIndex);
-          ka = static_cast<unsigned>(ka) >= static_cast<unsigned>(T) ? 0 : ka;
-          kb2 = static_cast<unsigned>(kb2) >= static_cast<unsigned>(T) ? 0 : kb2;
+          ka = 0;
         }
         int *ks = kidx + (g & 3) * 128;
-        ks[pt] = ka;
-        if (pt < 32) ks[pt + 96] = kb2;
-        mbar_arrive(kidx_bar);
-        if (!wait_warp(kidx_bar, kidx_phase & 1, p.status, abort_flag)) return false;
-        ++kidx_phase;
-        if (g + 1 < total) load_keys(g + 1, ka, kb2);
+        if (kload) ks[krow] = ka;
+        __syncwarp();
+        if (g + 1 < total) load_keys(g + 1, ka);
         gather(p.k_ptr, sK + s * kTileBytes, ks, hh);
         cp_async_arrive_noinc(&k_full[s]);
       } else if (pw == 0 && lane == 0) {
