@@ -396,10 +396,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence32(t + 32);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const uint32_t lv = live_bits((half ^ 1) * 2 + c);
+            const uint32_t lv = live_bits((half ^ 1) * 2 + c);   // the same in every lane
+            if (lv == 0xffffffffu) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              mxp[e & 3] = fmaxf(mxp[e & 3], ((lv >> e) & 1u) ? t[32 * c + e] : -INFINITY);
+              for (int e = 0; e < 32; ++e) mxp[e & 3] = fmaxf(mxp[e & 3], t[32 * c + e]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                mxp[e & 3] = fmaxf(mxp[e & 3], ((lv >> e) & 1u) ? t[32 * c + e] : -INFINITY);
+            }
           }
         }
         float sv[64];
