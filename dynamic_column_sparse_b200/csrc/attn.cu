@@ -10,8 +10,8 @@
 // loads. Warp 8 issues the tcgen05 MMAs: S = Q K^T into one of two TMEM
 // buffers, then O += P V with P read from TMEM and V from shared memory.
 // Warps 0-7 run the online softmax, two warps per TMEM lane quadrant (32
-// query rows), each on one 64-key half of S: both read the whole row to take
-// its maximum, exponentiate their half into P (bf16 pairs stored into one of
+// query rows), each on one 64-key half of S: they exchange their halves'
+// maxima for the row maximum, exponentiate their half into P (bf16 pairs stored into one of
 // two TMEM buffers with tcgen05.st) and rescale O in TMEM only when the row
 // maximum grows by more than 2^8. S of chunk i+1 is computed while the
 // softmax of chunk i runs. Logits are kept in log2 units (scale * log2 e).
@@ -34,7 +34,8 @@ constexpr uint32_t kTileBytes = 32768;   // one 128 x 128 bf16 operand tile (two
 constexpr float kRescaleLog2 = 8.0f;     // O and l are rescaled only when the row max grows by more than 2^8
 
 // Shared memory: Q | K[2] | V[2] | barriers | key-index ring [4][128] |
-// row-sum exchange [2][2][128] | key mask (complement pass).
+// row-sum exchange [2][2][128] | row-maximum exchange [2][2][128] | key mask
+// (complement pass) or merge buffers (delta pass).
 struct AttnCfg {
   static constexpr uint32_t kQOff = 0;
   static constexpr uint32_t kKOff = kTileBytes;
@@ -42,7 +43,8 @@ struct AttnCfg {
   static constexpr uint32_t kBarOff = kVOff + 2 * kTileBytes;
   static constexpr uint32_t kIdxOff = kBarOff + 256;
   static constexpr uint32_t kXsumOff = kIdxOff + 4 * 128 * 4;
-  static constexpr uint32_t kMaskOff = kXsumOff + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kXmaxOff = kXsumOff + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kMaskOff = kXmaxOff + 2 * 2 * 128 * 4;
 };
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
@@ -87,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [4][128] selected keys of chunk g at g & 3
   float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
+  float *xmax = reinterpret_cast<float *>(smem + C::kXmaxOff);   // [2][2][128] partial row maxima by chunk parity
   uint32_t *mask = reinterpret_cast<uint32_t *>(smem + C::kMaskOff);
   float *ebuf = reinterpret_cast<float *>(smem + C::kMaskOff);      // delta pass: [8 warps][32][36] merge buffer
 
@@ -381,32 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (MODE == kAttnComplement && lim > 0) m &= ~mask[base >> 5];
           return m;
         };
-        // The row maximum over all 128 keys: this warp also reads the other
-        // half's S columns (only to take their maximum), so both warps of the
-        // row reach the same maximum and the same rescale decision without
-        // exchanging anything.
+        // The row maximum over all 128 keys: each warp takes the maximum of its
+        // half and the two warps of the quadrant exchange them through shared
+        // memory, so both reach the same maximum and the same rescale decision.
         float mxp[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) mxp[u] = -INFINITY;
-        {
-          float t[64];
-          tmem_ld32_async(tmem + lane_off + s * 128 + (half ^ 1) * 64, t);
-          tmem_ld32_async(tmem + lane_off + s * 128 + (half ^ 1) * 64 + 32, t + 32);
-          tmem_wait_ld_regs(t);
-          reg_fence32(t + 32);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint32_t lv = live_bits((half ^ 1) * 2 + c);   // the same in every lane
-            if (lv == 0xffffffffu) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) mxp[e & 3] = fmaxf(mxp[e & 3], t[32 * c + e]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                mxp[e & 3] = fmaxf(mxp[e & 3], ((lv >> e) & 1u) ? t[32 * c + e] : -INFINITY);
-            }
-          }
-        }
         float sv[64];
         tmem_ld32_async(tmem + lane_off + s * 128 + half * 64, sv);
         tmem_ld32_async(tmem + lane_off + s * 128 + half * 64 + 32, sv + 32);
@@ -423,7 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int e = 0; e < 64; ++e) mxp[e & 3] = fmaxf(mxp[e & 3], sv[e]);
-        const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * sl2;
+        float mh = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+        {
+          float *xm = xmax + (g & 1) * 256;
+          xm[half * 128 + r] = mh;
+          if (!pair_sync()) {
+            ok = false;
+            break;
+          }
+          mh = fmaxf(mh, xm[(half ^ 1) * 128 + r]);
+        }
+        const float mx = mh * sl2;
         const float m_new = fmaxf(m_used, mx);
         // lazy rescale: only when the max grows by more than 2^8 over the one in use
         const bool need = m_used != -INFINITY && m_new > m_used + kRescaleLog2;

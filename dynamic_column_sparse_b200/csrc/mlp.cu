@@ -403,6 +403,366 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
   if (warp == kMmaWarp) tmem_dealloc(tmem, 2 * BT);
 }
 
+// Kernel 1 for 128-token blocks, wide form: tiles (token block b, chunk of
+// N = 256 hidden columns). The MMA computes D[token][col] with the x tile as
+// operand A (M = 128 tokens) and the 256 W1^T rows as operand B (N = 256), so
+// each K step reads 48 KB of operands from shared memory for 4.2 MFLOP and
+// every x tile serves 256 columns. One CTA per SM: warps 0-7 gather (sparse
+// step), warp 8 issues the MMAs into two TMEM accumulators of 256 columns,
+// warps 9-12 run the epilogue, warp 13 loads x (and, on a refresh, the
+// consecutive W1^T rows) by TMA. The epilogue warp of lane quadrant q owns
+// tokens 32q .. 32q + 31; it turns each 32 x 32 accumulator chunk around in a
+// padded shared buffer so that a thread holds one column's 32 tokens, and
+// moves the activation-cache and delta runs of those tokens (64 bytes per
+// column) through a second buffer as whole runs. The refresh uses this form;
+// on a sparse step the two-CTA form above measured as fast or faster (FLUX.1-dev
+// layer: 137 against 140 us), so the sparse step keeps that one.
+template <int N>
+struct UpWideCfg : Roles<8, 4> {
+  static constexpr int kN = N;                         // selected columns per tile
+  static constexpr uint32_t kTmemCols = 512;           // two accumulators of kN columns, allocated as a power of two
+  static_assert(2 * N <= 512, "two accumulators must fit in TMEM");
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kABytes = 128 * 128;       // x: 128 tokens x 64 bf16
+  static constexpr uint32_t kBBytes = kN * 128;        // gathered W1^T: kN rows x 64 bf16
+  static constexpr uint32_t kBOff = kStages * kABytes;
+  static constexpr uint32_t kPartOff = kBOff + kStages * kBBytes;   // refresh: [4][kN] partial column scores
+  static constexpr uint32_t kBarOff = kPartOff + 4 * kN * 4;
+  static constexpr uint32_t kTrOff = kBarOff + 1024;                // per epilogue warp: 32 x 33 fp32
+  static constexpr uint32_t kTbOff = kTrOff + kEpiWarps * 32 * 33 * 4;   // per epilogue warp: 32 x 80 B
+  static constexpr uint32_t kSmem = 1024 + kTbOff + kEpiWarps * 32 * 80;
+};
+
+template <int N, bool DENSE>
+__global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
+    mlp_up_wide_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
+                       const MlpUpParams p) {
+  using C = UpWideCfg<N>;
+  static_assert(!DENSE || N % 128 == 0, "a refresh loads the consecutive W1^T rows in boxes of 128");
+  constexpr int BT = 128, kN = C::kN, S = C::kStages;
+  constexpr int kProducers = C::kProducers, kMmaWarp = C::kMmaWarp, kTmaWarp = C::kTmaWarp;
+  constexpr int kRowIters = kN * 8 / kProducers;   // gathered 16-byte pieces of a stage per producer thread
+  constexpr int kRowStep = kProducers / 8;         // rows covered by one pass of all producer threads
+  constexpr uint32_t kIdesc = idesc_bf16(128, kN, false, false);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align_up<1024>(smem_raw);
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + C::kBOff;
+  float *part = reinterpret_cast<float *>(smem + C::kPartOff);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+  uint64_t *empty = full + S;
+  uint64_t *acc_full = empty + S;     // [2]
+  uint64_t *acc_empty = acc_full + 2; // [2]
+  uint64_t *part_bar = acc_empty + 2; // refresh: the four token quarters' partial scores are written / read
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(part_bar + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*(volatile int *)p.status != kDevOk) return;
+  const bool sparse = p.mode == kUpDelta;
+  const int kcols = sparse ? p.k : p.H;                 // columns of the block that are computed
+  const int nch = (kcols + kN - 1) / kN;
+  const int ntiles = p.nb * nch;
+  const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
+                           ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                           : 0;
+  const int nk = p.D / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], DENSE ? 1 : 1 + kProducers);   // the TMA thread (+ every gathering thread)
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 32 * C::kEpiWarps);
+    }
+    mbar_init(part_bar, 32 * C::kEpiWarps);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x == kTmaWarp * 32) {
+    prefetch_tmap(&tm_w1t);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < C::kProdWarps) {
+    // gathered W1^T rows: thread pt moves 16-byte piece (pt & 7) of rows
+    // i * kRowStep + (pt >> 3), i = 0 .. kRowIters - 1
+    if (!DENSE) {
+      const int pt = threadIdx.x;
+      uint32_t dst_off[kRowIters];
+#pragma unroll
+      for (int i = 0; i < kRowIters; ++i) dst_off[i] = sw128_offset(i * kRowStep + (pt >> 3), pt & 7);
+      // this thread's selected columns of the CTA's tile tl, loaded one tile
+      // ahead and range-checked when they are used
+      auto load_rows = [&](int tl, int *c) {
+        const int tile = blockIdx.x + tl * gridDim.x;
+        const int chunk = tile / p.nb, b = tile % p.nb;
+#pragma unroll
+        for (int i = 0; i < kRowIters; ++i)
+          c[i] = tl < my_tiles ? __ldg(p.idx + static_cast<size_t>(b) * p.k +
+                                      min(chunk * kN + i * kRowStep + (pt >> 3), p.k - 1))
+                               : 0;
+      };
+      int nxt[kRowIters];
+      load_rows(0, nxt);
+      const uint32_t b_base = smem_u32(sB);
+      int kg = 0;
+      bool ok = true;
+      for (int tl = 0; tl < my_tiles && ok; ++tl) {
+        const uint16_t *src_row[kRowIters];
+#pragma unroll
+        for (int i = 0; i < kRowIters; ++i) {
+          int c = nxt[i];
+          if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights
+            atomicCAS(p.status, kDevOk, kDevBadIndex);
+            c = 0;
+          }
+          src_row[i] = p.w1t + static_cast<size_t>(c) * p.D + (pt & 7) * 8;
+        }
+        load_rows(tl + 1, nxt);
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          if (!wait_warp(&empty[s], ((kg / S) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t stage = b_base + s * C::kBBytes;
+#pragma unroll
+          for (int i = 0; i < kRowIters; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
+          cp_async_arrive_noinc(&full[s]);
+        }
+      }
+    }
+  } else if (warp == kTmaWarp) {
+    // x tiles (and, on a refresh, the consecutive W1^T rows) by TMA
+    int kg = 0;
+    bool ok = true;
+    for (int tl = 0; tl < my_tiles && ok; ++tl) {
+      const int tile = blockIdx.x + tl * gridDim.x;
+      const int chunk = tile / p.nb, b = tile % p.nb;
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int s = kg % S;
+        if (!wait_warp(&empty[s], ((kg / S) & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], DENSE ? C::kABytes + C::kBBytes : C::kABytes);
+          tma_load_2d(sA + s * C::kABytes, &tm_x, &full[s], kb * kBK, b * BT);
+          if (DENSE) {
+#pragma unroll
+            for (int h = 0; h < kN / 128; ++h)
+              tma_load_2d(sB + s * C::kBBytes + h * 16384, &tm_w1t, &full[s], kb * kBK, chunk * kN + h * 128);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    int kg = 0;
+    bool ok = true;
+    for (int tl = 0; tl < my_tiles && ok; ++tl) {
+      const int ab = tl & 1;
+      const uint32_t tacc = tmem + ab * kN;
+      if (!wait_warp(&acc_empty[ab], ((tl >> 1) & 1) ^ 1, p.status, abort_flag)) break;
+      tc_fence_after();
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int s = kg % S;
+        if (!wait_warp(&full[s], (kg / S) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (!DENSE) fence_async_smem();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sA + s * C::kABytes);
+          const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16(tacc, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), kIdesc,
+                      (kb | kk) != 0);
+          umma_commit(&empty[s]);
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) umma_commit(&acc_full[ab]);
+      __syncwarp();
+    }
+  } else {
+    // epilogue: warp of lane quadrant q = tokens 32q .. 32q + 31, 32 columns at a time
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const bool first = p.mode == kUpRefreshFirst;
+    float *tr = reinterpret_cast<float *>(smem + C::kTrOff) + (warp - C::kEpiWarp0) * (32 * 33);
+    uint8_t *tb = smem + C::kTbOff + (warp - C::kEpiWarp0) * (32 * 80);
+    const int ck = lane & 3, cq = lane >> 2;   // run piece and column (8 i + cq) this lane moves
+    uint32_t part_phase = 0;
+    for (int tl = 0; tl < my_tiles; ++tl) {
+      const int tile = blockIdx.x + tl * gridDim.x;
+      const int chunk = tile / p.nb, b = tile % p.nb;
+      const int ab = tl & 1;
+      const int nvalid = min(BT, p.T - b * BT);
+      // hidden unit of column j = chunk * kN + 32 cc + lane, for all chunks cc
+      // of the tile at once (one load latency), range-checked here
+      int c_of[kN / 32];
+#pragma unroll
+      for (int cc = 0; cc < kN / 32; ++cc) {
+        const int j = chunk * kN + cc * 32 + lane;
+        if (sparse) {
+          c_of[cc] = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
+        } else {
+          c_of[cc] = min(j, p.H - 1);
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < kN / 32; ++cc) {
+        if (static_cast<unsigned>(c_of[cc]) >= static_cast<unsigned>(p.H)) {  // never address outside the cache
+          atomicCAS(p.status, kDevOk, kDevBadIndex);
+          c_of[cc] = 0;
+        }
+      }
+      // old activations of tokens 32q .. 32q + 31 for the columns 8 i + cq of chunk cc, and the bias
+      const size_t a_off = static_cast<size_t>(b) * p.H * BT + q * 32 + ck * 8;
+      auto load_old = [&](int cc, uint4 (&pre)[4], float &bias) {
+        const int c = c_of[cc];
+        const bool need_old = chunk * kN + cc * 32 + lane < kcols && !(first && !sparse);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int ci = __shfl_sync(0xffffffffu, c, 8 * i + cq);
+          const bool ni = __shfl_sync(0xffffffffu, need_old, 8 * i + cq);
+          pre[i] = ni ? *reinterpret_cast<const uint4 *>(p.a_cache + a_off + static_cast<size_t>(ci) * BT)
+                      : make_uint4(0, 0, 0, 0);
+        }
+        bias = bf16_bits_to_f32(__ldg(p.b1 + c));
+      };
+      uint4 pre[4];
+      float bias;
+      load_old(0, pre, bias);
+      if (!wait_warp(&acc_full[ab], (tl >> 1) & 1, p.status, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < kN / 32; ++cc) {
+        const int c = c_of[cc];
+        const bool valid_j = chunk * kN + cc * 32 + lane < kcols;
+        // old activations into the run buffer, then this thread's column out of it;
+        // the next chunk's are requested right away
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4 *>(tb + (8 * i + cq) * 80 + ck * 16) = pre[i];
+        const float bias_c = bias;
+        if (cc + 1 < kN / 32) load_old(cc + 1, pre, bias);
+        __syncwarp();
+        uint4 oldw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) oldw[u] = *reinterpret_cast<const uint4 *>(tb + lane * 80 + u * 16);
+        // accumulator chunk: lane = token, 32 columns; turned around so that lane = column
+        {
+          float acc[32];
+          tmem_ld32(tmem + lane_off + ab * kN + cc * 32, acc);
+          if (cc == kN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tr[lane * 33 + i] = acc[i];
+        }
+        __syncwarp();
+        float v[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = tr[t * 33 + lane];
+        const uint16_t *old = reinterpret_cast<const uint16_t *>(oldw);
+        float score = 0.f;
+        uint32_t na[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          uint16_t nab[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const float a = gelu_tanh(v[i + u] + bias_c);
+            const bool tok = q * 32 + i + u < nvalid;
+            nab[u] = tok ? f32_to_bf16_bits(a) : old[i + u];
+            if (!sparse) score += tok ? fabsf(first ? a : a - bf16_bits_to_f32(old[i + u])) : 0.f;
+          }
+          na[i / 2] = static_cast<uint32_t>(nab[0]) | (static_cast<uint32_t>(nab[1]) << 16);
+        }
+        // new activations back out as whole runs
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4 *>(tb + lane * 80 + u * 16) = make_uint4(na[4 * u], na[4 * u + 1], na[4 * u + 2], na[4 * u + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int ci = __shfl_sync(0xffffffffu, c, 8 * i + cq);
+          if (chunk * kN + cc * 32 + 8 * i + cq < kcols)
+            *reinterpret_cast<uint4 *>(p.a_cache + a_off + static_cast<size_t>(ci) * BT) =
+                *reinterpret_cast<const uint4 *>(tb + (8 * i + cq) * 80 + ck * 16);
+        }
+        if (sparse) {
+          // delta = bf16(new) - old for real tokens of a selected column, else 0;
+          // rows up to the padded width are written, none beyond it
+          const uint16_t *nw = reinterpret_cast<const uint16_t *>(na);
+          uint32_t dl[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            uint16_t dlb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const bool tok = q * 32 + i + u < nvalid;
+              dlb[u] = (valid_j && tok) ? f32_to_bf16_bits(bf16_bits_to_f32(nw[i + u]) - bf16_bits_to_f32(old[i + u]))
+                                        : static_cast<uint16_t>(0);
+            }
+            dl[i / 2] = static_cast<uint32_t>(dlb[0]) | (static_cast<uint32_t>(dlb[1]) << 16);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4 *>(tb + lane * 80 + u * 16) = make_uint4(dl[4 * u], dl[4 * u + 1], dl[4 * u + 2], dl[4 * u + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int jr = chunk * kN + cc * 32 + 8 * i + cq;
+            if (jr < p.k_pad)
+              *reinterpret_cast<uint4 *>(p.delta + (static_cast<size_t>(b) * p.k_pad + jr) * BT + q * 32 + ck * 8) =
+                  *reinterpret_cast<const uint4 *>(tb + (8 * i + cq) * 80 + ck * 16);
+          }
+        } else {
+          part[q * kN + cc * 32 + lane] = score;
+        }
+        __syncwarp();  // the buffers take the next chunk
+      }
+      if (!sparse) {
+        // column score = the four token quarters' partial sums, added in a fixed order
+        mbar_arrive(part_bar);
+        if (!wait_warp(part_bar, part_phase & 1, p.status, abort_flag)) break;
+        ++part_phase;
+        for (int col = (warp - C::kEpiWarp0) * 32 + lane; col < kN; col += 32 * C::kEpiWarps) {
+          const int j = chunk * kN + col;
+          if (j < kcols)
+            p.scores[static_cast<size_t>(b) * p.H + j] =
+                ((part[col] + part[kN + col]) + part[2 * kN + col]) + part[3 * kN + col];
+        }
+        mbar_arrive(part_bar);   // the partials have been read: the next tile may overwrite them
+        if (!wait_warp(part_bar, part_phase & 1, p.status, abort_flag)) break;
+        ++part_phase;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
+}
+
 template <int BN>
 struct DownCfg : Roles<8, 4> {   // eight gathering warps: the W2 stream is bound by cp.async issue per warp
   static constexpr int kCtasPerSm = 1;
@@ -717,6 +1077,21 @@ cudaError_t launch_up_t(const MlpUpParams &p, const CUtensorMap &w, const CUtens
   return cudaGetLastError();
 }
 
+template <int N, bool DENSE>
+cudaError_t launch_up_wide(const MlpUpParams &p, const CUtensorMap &w, const CUtensorMap &x, cudaStream_t s) {
+  using C = UpWideCfg<N>;
+  cudaError_t e = set_smem(mlp_up_wide_kernel<N, DENSE>, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int kcols = p.mode == kUpDelta ? p.k : p.H;
+  const int64_t tiles = static_cast<int64_t>(p.nb) * ((kcols + C::kN - 1) / C::kN);
+  const int64_t grid = std::min<int64_t>(tiles, sms);
+  mlp_up_wide_kernel<N, DENSE><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, s>>>(w, x, p);
+  return cudaGetLastError();
+}
+
 template <int BT, int BN, bool DENSE>
 cudaError_t launch_down_t(const MlpDownParams &p, const CUtensorMap &a, const CUtensorMap &w, cudaStream_t s) {
   using C = DownCfg<BN>;
@@ -745,7 +1120,7 @@ cudaError_t launch_down_bn(const MlpDownParams &p, const CUtensorMap &a, const C
 cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s) {
   if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
   const bool dense = p.mode != kUpDelta;
-  if (p.Bt == 128) return dense ? launch_up_t<128, true>(p, tm_w1t, tm_x, s) : launch_up_t<128, false>(p, tm_w1t, tm_x, s);
+  if (p.Bt == 128) return dense ? launch_up_wide<256, true>(p, tm_w1t, tm_x, s) : launch_up_t<128, false>(p, tm_w1t, tm_x, s);
   if (p.Bt == 64) return dense ? launch_up_t<64, true>(p, tm_w1t, tm_x, s) : launch_up_t<64, false>(p, tm_w1t, tm_x, s);
   return cudaErrorInvalidValue;
 }
