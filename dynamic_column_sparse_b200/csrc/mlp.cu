@@ -23,7 +23,12 @@
 //
 // Each kernel keeps two shared-memory rings: one for the gathered operand
 // (filled by the cp.async producer warps) and one for the operand that
-// arrives by tiled TMA. The warp roles are listed with `Roles` below.
+// arrives by tiled TMA. The warp roles are listed with `Roles` below. Data
+// written by cp.async must pass a generic-to-async proxy fence before the
+// tensor core reads it; in mlp_up the TMA warp takes that fence for each
+// gathered stage and hands the stage on through a second barrier, because the
+// fence stalls whichever warp executes it and the MMA warp is mlp_up's
+// critical path (mlp_down's MMA warp takes it itself at no measurable cost).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -102,6 +107,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
   uint64_t *part_bar = acc_empty + 2;  // refresh: both token halves of every column have their partial score
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(part_bar + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint64_t *a_ready = part_bar + 2;    // [SA] sparse step: a gathered stage is ordered for the tensor core
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*(volatile int *)p.status != kDevOk) return;
@@ -126,6 +132,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       mbar_init(&acc_empty[s], kEpiThreads);
     }
     mbar_init(part_bar, kEpiThreads);
+    for (int s = 0; s < SA; ++s) mbar_init(&a_ready[s], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -220,6 +227,25 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
           tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kBK, b * BT);
         }
         __syncwarp();
+        if (!DENSE && kg >= 1) {
+          // the previous gathered stage has landed: order it for the tensor core here,
+          // off the MMA warp
+          const int r = kg - 1;
+          if (!wait_warp(&a_full[r % SA], (r / SA) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          fence_async_smem();
+          if (lane == 0) mbar_arrive(&a_ready[r % SA]);
+          __syncwarp();
+        }
+      }
+    }
+    if (!DENSE && ok && kg >= 1) {
+      const int r = kg - 1;
+      if (wait_warp(&a_full[r % SA], (r / SA) & 1, p.status, abort_flag)) {
+        fence_async_smem();
+        if (lane == 0) mbar_arrive(&a_ready[r % SA]);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -232,12 +258,11 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       tc_fence_after();
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         const int sa = kg % SA, sb = kg % SB;
-        if (!wait_warp(&a_full[sa], (kg / SA) & 1, p.status, abort_flag) ||
+        if (!wait_warp(DENSE ? &a_full[sa] : &a_ready[sa], (kg / SA) & 1, p.status, abort_flag) ||
             !wait_warp(&b_full[sb], (kg / SB) & 1, p.status, abort_flag)) {
           ok = false;
           break;
         }
-        if (!DENSE) fence_async_smem();
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
