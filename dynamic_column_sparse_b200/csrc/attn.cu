@@ -764,6 +764,7 @@ template <int MODE>
 uint32_t attn_smem(int64_t T) {
   const uint32_t mask_bytes = MODE == kAttnComplement ? ((static_cast<uint32_t>(T) + 31) / 32) * 4 : 0;
   const uint32_t merge_bytes = MODE == kAttnDelta ? 8 * 32 * 36 * 4 : 0;
+  static_assert(1024 + AttnCfg::kMaskOff + 8 * 32 * 36 * 4 <= 232448, "delta pass over one CTA's shared memory");
   return 1024 + AttnCfg::kMaskOff + mask_bytes + merge_bytes;
 }
 

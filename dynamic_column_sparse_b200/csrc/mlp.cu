@@ -1,11 +1,12 @@
 // mlp.cu - gathered-column MLP kernels of the sparse delta step and the refresh.
 //
-// Kernel 1 (mlp_up): tiles (token block b, chunk of 128 selected hidden
-// columns), walked by persistent CTAs. The 128 selected rows of W1^T are
-// gathered into a 128-byte-swizzled shared tile by four producer warps with
-// 16-byte cp.async (each warp instruction moves four whole 128-byte row
-// segments); on a refresh, where the rows are consecutive, one TMA tile load
-// brings them instead. The token block of x arrives by a tiled TMA load. One
+// Kernel 1 (mlp_up, the sparse step and the refresh of 64-token blocks):
+// tiles (token block b, chunk of 128 selected hidden columns), walked by
+// persistent CTAs, two per SM. The 128 selected rows of W1^T are gathered
+// into a 128-byte-swizzled shared tile by four producer warps with 16-byte
+// cp.async (each warp instruction moves four whole 128-byte row segments); on
+// a refresh, where the rows are consecutive, one TMA tile load brings them
+// instead. (The refresh of 128-token blocks runs the wide form further down.) The token block of x arrives by a tiled TMA load. One
 // thread issues tcgen05 bf16 MMAs accumulating D[col][token] in one of two
 // TMEM accumulators. Each epilogue thread owns one hidden column (one TMEM
 // lane); the activation cache runs a_cache[b][c][..] and the delta rows are
@@ -73,6 +74,7 @@ struct UpCfg : Roles<4, 4> {
   static constexpr uint32_t kTbBytes = 32 * 80;  // per epilogue warp: 32 columns x 32 tokens bf16, rows padded to 80 B
   static constexpr uint32_t kEpiOff = kBarOff + 1024;
   static constexpr uint32_t kSmem = 1024 + kEpiOff + kEpiWarps * kTbBytes;
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "two CTAs must fit in one SM's shared memory");
 };
 
 // Persistent: CTA c handles tiles c, c + gridDim.x, ... where tile = chunk * nb
@@ -456,6 +458,7 @@ struct UpWideCfg : Roles<8, 4> {
   static constexpr uint32_t kTrOff = kBarOff + 1024;                // per epilogue warp: 32 x 33 fp32
   static constexpr uint32_t kTbOff = kTrOff + kEpiWarps * 32 * 33 * 4;   // per epilogue warp: 32 x 80 B
   static constexpr uint32_t kSmem = 1024 + kTbOff + kEpiWarps * 32 * 80;
+  static_assert(kSmem <= 232448, "over the shared memory of one CTA");
 };
 
 template <int N, bool DENSE>
@@ -800,6 +803,7 @@ struct DownCfg : Roles<8, 4> {   // eight gathering warps: the W2 stream is boun
   static constexpr uint32_t kBarOff = kBOff + kStagesB * kBBytes;
   static constexpr uint32_t kEpiOff = kBarOff + 1024;   // per epilogue warp: 32 x 33 fp32 transpose buffer
   static constexpr uint32_t kSmem = 1024 + kEpiOff + kEpiWarps * 32 * 33 * 4;
+  static_assert(kSmem <= 232448, "over the shared memory of one CTA");
 };
 
 // Persistent: CTA c handles tiles c, c + gridDim.x, ...; the two TMEM
