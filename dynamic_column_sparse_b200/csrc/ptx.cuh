@@ -1,5 +1,6 @@
-// ptx.cuh - thin inline-PTX wrappers for sm_100a: mbarriers, TMA (tile and
-// gather4), tcgen05 (TMEM alloc, MMA, commit, loads) and the UMMA descriptors.
+// ptx.cuh - thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads,
+// cp.async, tcgen05 (TMEM alloc, MMA, commit, loads, stores) and the UMMA
+// descriptors.
 #pragma once
 
 #include <cuda.h>
@@ -88,11 +89,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *s
   }
 }
 
-// Barrier over `count` threads (a multiple of 32) of the CTA, id 1..15.
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ----------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *tm) {
@@ -119,17 +115,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, ui
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-// Four rows y0..y3 of a 2-D tensor, columns [x, x + box width), into four
-// consecutive box rows at dst. The tensor map's box must be one row high.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *tm, uint64_t *bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
 
@@ -200,8 +185,6 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
