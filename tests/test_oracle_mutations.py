@@ -172,6 +172,63 @@ def _delta_compact_unweighted(q, k, v, idx, lse_c, o_c, scale, Bt):
     return out
 
 
+def _k_round_up(n, density_permille):
+    return -((-int(n) * int(density_permille)) // 1000)
+
+
+def _dense_mlp_no_b2(x, W1, b1, W2, b2):
+    a = OC.gelu_tanh(x @ W1 + b1[None, :])
+    return a, a @ W2
+
+
+def _finish_unnormalised(p):
+    m, l, acc = p
+    return np.asarray(acc, dtype=np.float64)
+
+
+def _attn_delta_ignores_cache(q, k, v, idx, m_c, l_c, acc_c, scale, Bt):
+    h, T, d = q.shape
+    out = np.zeros((h, T, d))
+    for hh in range(h):
+        for b, r0, r1 in OC.blocks(T, Bt):
+            S = np.asarray(idx[hh][b], dtype=np.int64)
+            out[hh, r0:r1] = OC.finish(OC.attn_partial(q[hh, r0:r1], k[hh, S], v[hh, S], scale))
+    return out
+
+
+def _dense_attention_lse_without_max(q, k, v, scale):
+    h, T, d = q.shape
+    O = np.zeros((h, T, d))
+    lse = np.zeros((h, T))
+    for hh in range(h):
+        m, l, acc = OC.attn_partial(q[hh], k[hh], v[hh], scale)
+        O[hh] = acc / l[:, None]
+        lse[hh] = np.log(l)
+    return O, lse
+
+
+def _mass_rows_no_scale(q_rows, k, scale):
+    s = q_rows @ k.T
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p.sum(axis=0)
+
+
+def _mlp_refresh_ignores_first_step(x, W1, b1, W2, b2, A_old, Bt, k, first_step):
+    a, y = OC.dense_mlp(x, W1, b1, W2, b2)
+    scores = OC.mlp_scores(a, A_old if A_old is not None else np.zeros_like(a), Bt, False)
+    return dict(a=a, y=y, scores=scores, idx=OC.topk_cols(OC.f32(scores), k))
+
+
+def _attn_refresh_smallest_mass(q, k, v, scale, Bt, kk):
+    O, lse = OC.dense_attention(q, k, v, scale)
+    mass = OC.attn_mass(q, k, scale, Bt)
+    h, nb, T = mass.shape
+    idx = OC.topk_cols(OC.f32(-mass.reshape(h * nb, T)), kk).reshape(h, nb, kk)
+    m_c, l_c, acc_c = OC.complement_partial(q, k, v, idx, scale, Bt)
+    return dict(O=O, lse=lse, mass=mass, idx=idx, m_c=m_c, l_c=l_c, acc_c=acc_c)
+
+
 MUTATIONS = {
     "gelu_tanh: cubic term dropped": ("gelu_tanh", _gelu_no_cubic),
     "gelu_tanh: sign of tanh flipped": ("gelu_tanh", _gelu_sign),
@@ -189,6 +246,14 @@ MUTATIONS = {
     "bf16_round: truncation instead of nearest-even": ("bf16_round", _bf16_truncate),
     "compact_partial: log of l dropped": ("compact_partial", _compact_no_log),
     "attn_delta_compact: cached weight e^lse dropped": ("attn_delta_compact", _delta_compact_unweighted),
+    "k_from_density: rounded up": ("k_from_density", _k_round_up),
+    "dense_mlp: bias b2 dropped": ("dense_mlp", _dense_mlp_no_b2),
+    "finish: not divided by l": ("finish", _finish_unnormalised),
+    "attn_delta: cached complement ignored": ("attn_delta", _attn_delta_ignores_cache),
+    "dense_attention: lse without the row maximum": ("dense_attention", _dense_attention_lse_without_max),
+    "attn_mass_rows: logit scale dropped": ("attn_mass_rows", _mass_rows_no_scale),
+    "mlp_refresh: first-step rule ignored": ("mlp_refresh", _mlp_refresh_ignores_first_step),
+    "attn_refresh: smallest mass selected": ("attn_refresh", _attn_refresh_smallest_mass),
 }
 
 

@@ -252,6 +252,22 @@ def test_mlp_refresh_selects_top_scores_and_rebuilds_cache():
         assert min(s[list(sel)]) >= max(s[[c for c in range(20) if c not in sel]])
 
 
+def test_mlp_refresh_first_step_scores_ignore_the_cache():
+    # a first step has no cache: the score of a column is the sum over the
+    # block's rows of |a|, written out term by term, whatever A_old holds
+    x, W1, b1, W2, b2 = _mlp_case(T=16)
+    r0 = O.mlp_refresh(x, W1, b1, W2, b2, np.zeros((16, 20)), Bt=8, k=5, first_step=True)
+    r1 = O.mlp_refresh(x, W1, b1, W2, b2, rng.standard_normal((16, 20)), Bt=8, k=5, first_step=True)
+    for r in (r0, r1):
+        for b in range(2):
+            for c in range(20):
+                want = 0.0
+                for row in range(8 * b, 8 * b + 8):
+                    want += abs(r["a"][row, c])
+                assert abs(r["scores"][b, c] - want) <= 1e-12 * max(1.0, want)
+    np.testing.assert_array_equal(r0["idx"], r1["idx"])
+
+
 # --------------------------------------------------------------------------- attention
 
 def _softmax_attention_brute(q, k, v, scale, keys=None):
