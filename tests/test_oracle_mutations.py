@@ -229,6 +229,15 @@ def _attn_refresh_smallest_mass(q, k, v, scale, Bt, kk):
     return dict(O=O, lse=lse, mass=mass, idx=idx, m_c=m_c, l_c=l_c, acc_c=acc_c)
 
 
+def _blocks_drop_short_tail(T, Bt):
+    return [(b, b * Bt, (b + 1) * Bt) for b in range(T // Bt)]
+
+
+def _bf16_decode_low_half(bits):
+    with np.errstate(invalid="ignore"):
+        return (np.asarray(bits, dtype=np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)
+
+
 MUTATIONS = {
     "gelu_tanh: cubic term dropped": ("gelu_tanh", _gelu_no_cubic),
     "gelu_tanh: sign of tanh flipped": ("gelu_tanh", _gelu_sign),
@@ -254,6 +263,8 @@ MUTATIONS = {
     "attn_mass_rows: logit scale dropped": ("attn_mass_rows", _mass_rows_no_scale),
     "mlp_refresh: first-step rule ignored": ("mlp_refresh", _mlp_refresh_ignores_first_step),
     "attn_refresh: smallest mass selected": ("attn_refresh", _attn_refresh_smallest_mass),
+    "blocks: short last block dropped": ("blocks", _blocks_drop_short_tail),
+    "bf16_decode: bits shifted by 15": ("bf16_decode", _bf16_decode_low_half),
 }
 
 
