@@ -28,6 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libchipmunk.so")
 
 OK = 0
+ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGNMENT, ERR_CUDA, ERR_DEVICE, ERR_UNSUPPORTED, ERR_WORKSPACE = 1, 2, 3, 4, 5, 6, 7
 OP_TOPK, OP_MLP_DELTA, OP_ATTN_DELTA, OP_REFRESH = 0, 1, 2, 3
 REFRESH_MLP, REFRESH_ATTN = 0, 1
 
@@ -159,7 +160,7 @@ def read_device_status(stream=None) -> int:
     lib = load_library()
     v = ctypes.c_int32(0)
     st = lib.chipmunk_read_device_status(ctypes.byref(v), _stream(stream))
-    if st not in (OK, 5):
+    if st not in (OK, ERR_DEVICE):
         _check(st)
     return int(v.value)
 
@@ -230,8 +231,9 @@ def mlp_delta(x, w1t, b1, w2, idx, a_cache, y_cache, out=None, Bt=128, workspace
 
 def mlp_delta_noalloc(x, w1t, b1, w2, idx, a_cache, y_cache, out=None, Bt=128, stream=None):
     """mlp_delta without caller scratch: for callers that cannot allocate device
-    memory. The library's fixed 64 MiB scratch array is shared by every call, so
-    calls must not overlap on the GPU; larger problems raise."""
+    memory. The library's fixed 64 MiB scratch array (reserved on a device at
+    this call's first use there) is shared by every call, so calls must not
+    overlap on the GPU; larger problems raise with status ERR_WORKSPACE."""
     lib = load_library()
     a = _mlp_args(x, w1t, b1, w2, None, idx, a_cache, y_cache, out, Bt, idx.shape[1])
     _check(lib.chipmunk_mlp_delta_noalloc(ctypes.byref(a), _stream(stream)))

@@ -11,6 +11,7 @@
 #include <string>
 
 #include "../../include/chipmunk.h"
+#include "abi_internal.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -234,6 +235,29 @@ chipmunk_status mlp_down_impl(const chipmunk_mlp_args *a, void *ws, int *status,
 
 }  // namespace
 
+namespace cm {
+
+chipmunk_status record_error(chipmunk_status st, const char *msg) { return fail(st, "%s", msg); }
+
+chipmunk_status mlp_delta_fixed_scratch(const chipmunk_mlp_args *a, size_t scratch_bytes,
+                                        chipmunk_status (*get_scratch)(void **), cudaStream_t s) {
+  CM_CHECK(check_mlp(a, false));
+  const size_t need = mlp_delta_ws(a);
+  if (need > scratch_bytes)
+    return fail(CHIPMUNK_ERR_WORKSPACE,
+                "chipmunk_mlp_delta_noalloc needs %zu bytes of scratch, more than its fixed %zu; "
+                "use chipmunk_mlp_delta with a caller workspace",
+                need, scratch_bytes);
+  int *status = nullptr;
+  CM_CHECK(device_setup(&status));
+  void *ws = nullptr;
+  CM_CHECK(get_scratch(&ws));
+  CM_CHECK(mlp_up_impl(a, ws, status, s));
+  return mlp_down_impl(a, ws, status, s);
+}
+
+}  // namespace cm
+
 extern "C" {
 
 const char *chipmunk_version(void) { return "0.1.0"; }
@@ -416,50 +440,6 @@ chipmunk_status chipmunk_scatter_cols(const void *packed, int64_t nb, int64_t H,
                                   static_cast<uint16_t *>(a_cache), status, static_cast<cudaStream_t>(stream)),
           "scatter launch");
   return CHIPMUNK_OK;
-}
-
-// Scratch of chipmunk_mlp_delta_noalloc: a fixed device array, one per device,
-// so that callers without an allocator can run the sparse MLP step. In host
-// code this name is a host-side stand-in; its device address comes from
-// cudaGetSymbolAddress below.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[CHIPMUNK_NOALLOC_SCRATCH_BYTES];
-
-static std::mutex g_noalloc_mu;
-static void *g_noalloc_ptr[kMaxDevices] = {};
-
-// One-time per-device look-up of the scratch array's device address, with
-// that device current (the caller's current device).
-static chipmunk_status noalloc_scratch(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(CHIPMUNK_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return CHIPMUNK_OK;
-}
-
-chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args *a, chipmunk_stream stream) {
-  CM_CHECK(check_mlp(a, false));
-  const size_t need = mlp_delta_ws(a);
-  if (need > CHIPMUNK_NOALLOC_SCRATCH_BYTES)
-    return fail(CHIPMUNK_ERR_WORKSPACE,
-                "chipmunk_mlp_delta_noalloc needs %zu bytes of scratch, more than its fixed %zu; "
-                "use chipmunk_mlp_delta with a caller workspace",
-                need, size_t(CHIPMUNK_NOALLOC_SCRATCH_BYTES));
-  int *status = nullptr;
-  CM_CHECK(device_setup(&status));
-  void *ws = nullptr;
-  CM_CHECK(noalloc_scratch(&ws));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CM_CHECK(mlp_up_impl(a, ws, status, s));
-  return mlp_down_impl(a, ws, status, s);
 }
 
 chipmunk_status chipmunk_selftest_bounded_wait(chipmunk_stream stream) {

@@ -303,14 +303,17 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       const int chunk = tile / p.nb, b = tile % p.nb;
       const int ab = tl & 1;
       const int j = chunk * 128 + r;
-      const bool valid_j = sparse ? (j < p.k) : (j < p.H);
+      bool valid_j = sparse ? (j < p.k) : (j < p.H);
       // column, bias and the cached activations are fetched before the accumulator is ready
       int c;
       if (sparse) {
         c = __ldg(p.idx + static_cast<size_t>(b) * p.k + min(j, p.k - 1));
-        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {  // never address outside the weights / cache
+        if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
+          // never address outside the weights / cache; the column is dropped: no cache
+          // write, and its delta row is zero so the down-projection adds nothing for it
           atomicCAS(p.status, kDevOk, kDevBadIndex);
           c = 0;
+          valid_j = false;
         }
       } else {
         c = min(j, p.H - 1);
@@ -652,18 +655,20 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
           c_of[cc] = min(j, p.H - 1);
         }
       }
+      uint32_t bad = 0;   // bit cc: this lane's column of chunk cc had an index out of range and is dropped
 #pragma unroll
       for (int cc = 0; cc < kN / 32; ++cc) {
         if (static_cast<unsigned>(c_of[cc]) >= static_cast<unsigned>(p.H)) {  // never address outside the cache
           atomicCAS(p.status, kDevOk, kDevBadIndex);
           c_of[cc] = 0;
+          bad |= 1u << cc;
         }
       }
       // old activations of tokens 32q .. 32q + 31 for the columns 8 i + cq of chunk cc, and the bias
       const size_t a_off = static_cast<size_t>(b) * p.H * BT + q * 32 + ck * 8;
       auto load_old = [&](int cc, uint4 (&pre)[4], float &bias) {
         const int c = c_of[cc];
-        const bool need_old = chunk * kN + cc * 32 + lane < kcols && !(first && !sparse);
+        const bool need_old = chunk * kN + cc * 32 + lane < kcols && !((bad >> cc) & 1u) && !(first && !sparse);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int ci = __shfl_sync(0xffffffffu, c, 8 * i + cq);
@@ -681,7 +686,7 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < kN / 32; ++cc) {
         const int c = c_of[cc];
-        const bool valid_j = chunk * kN + cc * 32 + lane < kcols;
+        const bool valid_j = chunk * kN + cc * 32 + lane < kcols && !((bad >> cc) & 1u);
         // old activations into the run buffer, then this thread's column out of it;
         // the next chunk's are requested right away
 #pragma unroll
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int ci = __shfl_sync(0xffffffffu, c, 8 * i + cq);
-          if (chunk * kN + cc * 32 + 8 * i + cq < kcols)
+          if (__shfl_sync(0xffffffffu, valid_j, 8 * i + cq))
             *reinterpret_cast<uint4 *>(p.a_cache + a_off + static_cast<size_t>(ci) * BT) =
                 *reinterpret_cast<const uint4 *>(tb + (8 * i + cq) * 80 + ck * 16);
         }

@@ -225,8 +225,14 @@ CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_down(const chipmunk_mlp_args *a,
  * allocation would synchronise the device. This call computes exactly what
  * chipmunk_mlp_delta computes, with the same arguments, but takes its delta
  * scratch from a fixed array inside the library instead of from the caller:
- *   - The array holds CHIPMUNK_NOALLOC_SCRATCH_BYTES (64 MiB). Every GPU that
- *     loads the library keeps it until the process exits.
+ *   - The array holds CHIPMUNK_NOALLOC_SCRATCH_BYTES (64 MiB). It is reserved
+ *     on a device when the part of the library that holds it is loaded there:
+ *     under CUDA's default lazy module loading, at this entry point's first
+ *     call on that device (no other entry point loads it); with
+ *     CUDA_MODULE_LOADING=EAGER, when the device's context is created. From
+ *     then on that device keeps it until the process exits. If the device has
+ *     no 64 MiB left at that moment, the first call returns CHIPMUNK_ERR_CUDA
+ *     and enqueues nothing.
  *   - Calls that need more (nb * round_up(k, 128) * Bt * 2 bytes; the
  *     FLUX.1-dev layer at 70% sparsity needs 32.3 MB) return
  *     CHIPMUNK_ERR_WORKSPACE and enqueue nothing.

@@ -129,3 +129,23 @@ def test_refresh_rejects_unknown_kind(cm):
     assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1
     r = cm.RefreshArgs(kind=cm.REFRESH_ATTN, scores=0)
     assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch(cm):
+    """The size check of the no-alloc entry point runs on the host, before any device call."""
+    lib = cm.load_library()
+    # nb * round_up(k,128) * Bt * 2 = 600 * 1024 * 128 * 2 bytes > 64 MiB
+    a = _mlp_args(cm, T=600 * 128, D=128, H=1024, Bt=128, k=1024, b2=0)
+    assert 600 * 1024 * 128 * 2 > cm.NOALLOC_SCRATCH_BYTES
+    assert lib.chipmunk_mlp_delta_noalloc(ctypes.byref(a), None) == cm.ERR_WORKSPACE
+    assert b"scratch" in lib.chipmunk_last_error()
+
+
+def test_status_constants_match_the_header(cm):
+    text = open(HEADER).read()
+    for name in ("OK", "ERR_INVALID_ARG", "ERR_SHAPE", "ERR_ALIGNMENT", "ERR_CUDA", "ERR_DEVICE", "ERR_UNSUPPORTED",
+                 "ERR_WORKSPACE"):
+        m = re.search(rf"#define CHIPMUNK_{name}\s+(\d+)", text)
+        assert m and int(m.group(1)) == getattr(cm, name), name
+    m = re.search(r"#define CHIPMUNK_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m and (int(m.group(1)) << int(m.group(2))) == cm.NOALLOC_SCRATCH_BYTES
