@@ -213,18 +213,23 @@ def finish(p):
     return np.where((l > 0)[:, None], acc / safe[:, None], 0.0)
 
 
-def attn_delta(q, k, v, idx, m_c, l_c, acc_c, scale, Bt):
+def attn_delta(q, k, v, idx, m_c, l_c, acc_c, scale, Bt, tiles=None):
     """Sparse attention step: recompute the selected keys, reuse the cached rest.
 
     For each head and query block the selected keys are attended with the
     current q, k, v and merged with the cached partial over the complementary
     keys (post: attention output as a sum of scaled rows of V, of which only a
-    subset is replaced on each step). Returns O [h][T][d].
+    subset is replaced on each step). Returns O [h][T][d]. With ``tiles`` (a
+    list of (head, query block) pairs) only those tiles are computed; the rest
+    of O is zero.
     """
     h, T, d = q.shape
     O = np.zeros((h, T, d))
+    todo = None if tiles is None else {(int(a), int(b)) for a, b in np.asarray(tiles).reshape(-1, 2)}
     for hh in range(h):
         for b, r0, r1 in blocks(T, Bt):
+            if todo is not None and (hh, b) not in todo:
+                continue
             S = np.asarray(idx[hh][b], dtype=np.int64)
             sel = attn_partial(q[hh, r0:r1], k[hh, S], v[hh, S], scale)
             cached = (m_c[hh, r0:r1], l_c[hh, r0:r1], acc_c[hh, r0:r1])

@@ -1,20 +1,29 @@
 """Mistakes planted in the oracle must be caught by its pins.
 
-Each mutation replaces one oracle function with a copy carrying a plausible
-error (a dropped term, a wrong sign or index, a transposed reduction, a wrong
-tie rule, a missing scale). The pin suite in test_oracle_pins.py is then run
-against the mutated oracle; at least one pin must fail. Everything runs on
-the CPU.
+Both oracles are mutated, one plausible error at a time (a dropped term, a
+wrong sign or index, a transposed reduction, a wrong tie rule, a missing
+scale):
+
+* the numpy oracle, by replacing one of its functions with a copy carrying
+  the error;
+* the C++ oracle, by rebuilding it from a copy of its source in which one
+  snippet is replaced (each snippet must occur exactly once).
+
+The pin suite in test_oracle_pins.py is then run against the mutated oracle;
+at least one pin must fail. The unmutated oracles must pass every pin.
+Everything runs on the CPU.
 """
+import concurrent.futures as cf
 import inspect
 import math
+import os
 
 import numpy as np
 import pytest
 
-import oracle
 import oracle.chipmunk_oracle as OC
 import test_oracle_pins as pins
+from oracle import cpp
 
 ORIG = {name: getattr(OC, name) for name in ("mlp_delta", "attn_partial")}
 
@@ -35,16 +44,20 @@ def _all_pins():
     return calls
 
 
-def _caught(monkeypatch, fname, mutant):
-    monkeypatch.setattr(OC, fname, mutant)
-    monkeypatch.setattr(oracle, fname, mutant)
+def _failed_pins(monkeypatch, impl):
+    monkeypatch.setattr(pins, "O", impl)
     failed = []
     for name, fn, kwargs in _all_pins():
         try:
             fn(**kwargs)
-        except AssertionError:
+        except (AssertionError, ValueError, IndexError):
             failed.append(name)
     return failed
+
+
+def _caught(monkeypatch, fname, mutant):
+    monkeypatch.setattr(OC, fname, mutant)
+    return _failed_pins(monkeypatch, OC)
 
 
 def _gelu_no_cubic(u):
@@ -277,3 +290,80 @@ def test_planted_mistake_is_caught(monkeypatch, what):
 
 def test_unmutated_oracle_passes_every_pin(monkeypatch):
     assert _caught(monkeypatch, "gelu_tanh", OC.gelu_tanh) == []
+
+
+# --------------------------------------------------------------------------- C++ oracle
+
+CPP_MUTATIONS = {
+    "gelu: cubic term dropped": ("(u + 0.044715 * u * u * u)", "(u)"),
+    "gelu: sign of tanh flipped": ("0.5 * u * (1.0 + std::tanh(", "0.5 * u * (1.0 - std::tanh("),
+    "mlp_delta: delta sign flipped": ("delta[r * k + j] = an - A_cache[(r0 + r) * H + c];",
+                                      "delta[r * k + j] = A_cache[(r0 + r) * H + c] - an;"),
+    "preactivation: bias b1 dropped": ("u[r] = acc[r] + b1[c];", "u[r] = acc[r];"),
+    "preactivation: first input feature skipped": ("  for (int64_t d = 0; d < D; ++d) {\n    const double *xd",
+                                                   "  for (int64_t d = 1; d < D; ++d) {\n    const double *xd"),
+    "mlp_delta: cache not written back": ("A_new[(r0 + r) * H + c] = an;", "(void)an;"),
+    "weighted_row_sums: last term of every chunk dropped": ("const int64_t j1 = std::min(j0 + kTerms, ncoef);",
+                                                            "const int64_t j1 = std::min(j0 + kTerms - 1, ncoef);"),
+    "weighted_row_sums: ragged output tail skipped": ("for (int64_t e = 0; e < nn; ++e) o[e] += coef[r * ldc + j] * rows[j][n0 + e];",
+                                                      "(void)nn;"),
+    "topk: ties to the higher index": ("[&](int64_t a, int64_t b) { return key[a] > key[b]; }",
+                                       "[&](int64_t a, int64_t b) { return key[a] != key[b] ? key[a] > key[b] : a > b; }"),
+    "topk: indices not ascending": ("std::sort(order.begin(), order.begin() + k);", ""),
+    "ordered_key: -0 not equal to +0": ("if (b == 0x80000000u) b = 0u;", ""),
+    "merge: weights inverted": ("const double w1 = (m1 == kNegInf) ? 0.0 : std::exp(m1 - mm);\n  const double w2 = (m2 == kNegInf) ? 0.0 : std::exp(m2 - mm);",
+                                "const double w1 = (m1 == kNegInf) ? 0.0 : std::exp(mm - m1);\n  const double w2 = (m2 == kNegInf) ? 0.0 : std::exp(mm - m2);"),
+    "partial: logit scale dropped": ("      s[j] *= scale;\n      mx = std::max(mx, s[j]);\n    }\n    double l = 0.0;\n    for (int64_t j = 0; j < m; ++j) {",
+                                     "      s[j] *= 1.0;\n      mx = std::max(mx, s[j]);\n    }\n    double l = 0.0;\n    for (int64_t j = 0; j < m; ++j) {"),
+    "mass: probabilities not normalised": ("out[j] += s[j] / l;", "out[j] += s[j];"),
+    "mass: logit scale dropped": ("      s[j] *= scale;\n      mx = std::max(mx, s[j]);\n    }\n    double l = 0.0;\n    for (int64_t j = 0; j < T; ++j) {",
+                                  "      s[j] *= 1.0;\n      mx = std::max(mx, s[j]);\n    }\n    double l = 0.0;\n    for (int64_t j = 0; j < T; ++j) {"),
+    "complement: selected keys kept": ("if (!selected[j]) keys.push_back(j);", "keys.push_back(j);"),
+    "mlp_scores: absolute value dropped": ("s += std::fabs(first_step ? a[r * H + c] : a[r * H + c] - A_cache[r * H + c]);",
+                                           "s += (first_step ? a[r * H + c] : a[r * H + c] - A_cache[r * H + c]);"),
+    "bf16_round: truncation instead of nearest-even": ("(static_cast<uint64_t>(u) + 0x7FFFu + lsb) >> 16",
+                                                       "(static_cast<uint64_t>(u) + 0u * lsb) >> 16"),
+    "compact_partial: log of l dropped": ("lse[i] = l[i] > 0 ? m[i] + std::log(l[i]) : kNegInf;",
+                                          "lse[i] = l[i] > 0 ? m[i] + l[i] : kNegInf;"),
+    "attn_delta_compact: cached weight e^lse dropped": ("merge_row(lse_c[row], 1.0,", "merge_row(0.0, 1.0,"),
+    "k_from_density: rounded up": ("return (n * permille) / 1000;", "return (n * permille + 999) / 1000;"),
+    "dense_mlp: bias b2 dropped": ("for (int64_t n = 0; n < D; ++n) y[r * D + n] += b2[n];", "(void)b2;"),
+    "finish: not divided by l": ("out[e] = l > 0 ? acc[e] / l : 0.0;", "out[e] = l > 0 ? acc[e] : 0.0;"),
+    "attn_delta: cached complement ignored": ("merge_row(m_c[row], l_c[row], acc_c + row * d,",
+                                              "merge_row(kNegInf, 0.0, acc_c + row * d,"),
+    "dense_attention: lse without the row maximum": ("lse[row] = m[i] + std::log(l[i]);", "lse[row] = std::log(l[i]);"),
+    "mlp_refresh: first-step rule ignored": ("or_mlp_scores(a, A_old, T, H, Bt, first_step, scores);",
+                                             "or_mlp_scores(a, A_old, T, H, Bt, 0, scores);"),
+    "attn_refresh: smallest mass selected": ("m32[i] = static_cast<float>(mass[i]);",
+                                             "m32[i] = static_cast<float>(-mass[i]);"),
+    "blocks: short last block dropped": ("int64_t block_count(int64_t T, int64_t Bt) { return (T + Bt - 1) / Bt; }",
+                                         "int64_t block_count(int64_t T, int64_t Bt) { return T / Bt; }"),
+    "bf16_decode: bits shifted by 15": ("static_cast<uint32_t>(bits) << 16;", "static_cast<uint32_t>(bits) << 15;"),
+}
+
+
+@pytest.fixture(scope="module")
+def cpp_mutants(tmp_path_factory):
+    """Every C++ mutant, built once (in parallel) into its own shared library."""
+    src = open(cpp.SRC).read()
+    out_dir = tmp_path_factory.mktemp("oracle_mutants")
+    jobs = {}
+    for i, (what, (old, new)) in enumerate(sorted(CPP_MUTATIONS.items())):
+        assert src.count(old) == 1, f"{what}: the snippet must occur exactly once in the source"
+        path = os.path.join(out_dir, f"m{i}.cpp")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        jobs[what] = path
+    with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        futs = {what: ex.submit(cpp.compile_source, p, p[:-4] + ".so") for what, p in jobs.items()}
+        return {what: f.result() for what, f in futs.items()}
+
+
+@pytest.mark.parametrize("what", sorted(CPP_MUTATIONS))
+def test_planted_mistake_in_cpp_oracle_is_caught(monkeypatch, cpp_mutants, what):
+    failed = _failed_pins(monkeypatch, cpp.CppOracle(cpp_mutants[what]))
+    assert failed, f"no pin caught: {what}"
+
+
+def test_unmutated_cpp_oracle_passes_every_pin(monkeypatch):
+    assert _failed_pins(monkeypatch, cpp.CppOracle(cpp.build())) == []

@@ -12,7 +12,23 @@ import os
 import numpy as np
 import pytest
 
-import oracle as O
+import oracle
+from oracle import numpy_oracle
+
+# The pins run against both oracles: the C++ one (oracle.default(), what the
+# GPU parity tests use) and its numpy cross-check. ``O`` is the one under test.
+IMPLS = {"cpp": oracle.default, "numpy": lambda: numpy_oracle}
+O = oracle
+
+
+@pytest.fixture(autouse=True, params=sorted(IMPLS))
+def impl(request):
+    global O
+    saved = O
+    O = IMPLS[request.param]()
+    yield request.param
+    O = saved
+
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 rng = np.random.default_rng(1234)
@@ -171,6 +187,65 @@ def test_dense_mlp_permutation_and_bias_structure():
         u = sum(x[t, d] * W1[d, c] for d in range(x.shape[1])) + b1[c]
         for n in range(W2.shape[1]):
             assert abs(y1[t, n] - _gelu_erf(u) * W2[c, n]) < 5e-4 * abs(W2[c, n]) + 1e-12
+
+
+def _mlp_brute(x, W1, b1, W2, b2, cols=None):
+    """gelu(x W1 + b1) W2 + b2 by plain loops, one term at a time (hidden units ``cols`` only, no
+    b2, when given)."""
+    T, D = x.shape
+    H = W1.shape[1]
+    cols = range(H) if cols is None else cols
+    y = np.zeros((T, W2.shape[1]))
+    a = {}
+    for t in range(T):
+        for c in cols:
+            u = 0.0
+            for d in range(D):
+                u += x[t, d] * W1[d, c]
+            u += b1[c]
+            a[t, c] = 0.5 * u * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+        for n in range(W2.shape[1]):
+            s = 0.0
+            for c in cols:
+                s += a[t, c] * W2[c, n]
+            y[t, n] = s
+    return a, y
+
+
+def test_dense_mlp_brute_force_at_a_moderate_size():
+    # 18 tokens, 40 features, 300 hidden units: more rows, features and hidden units than one
+    # group of the C++ oracle's loops handles at a time (16 rows, 16 outputs, 128 terms)
+    x, W1, b1, W2, b2 = _mlp_case(T=18, D=40, H=300, seed=7)
+    a, y = O.dense_mlp(x, W1, b1, W2, b2)
+    a_ref, y_ref = _mlp_brute(x, W1, b1, W2, b2)
+    for (t, c), v in a_ref.items():
+        assert abs(a[t, c] - v) <= 1e-13 * max(1.0, abs(v))
+    np.testing.assert_allclose(y, y_ref + b2, rtol=0, atol=1e-12)
+
+
+def test_mlp_delta_brute_force_at_a_moderate_size():
+    # 150 selected columns of 300 in blocks of 8 of 18 tokens: the update is the old output plus,
+    # per selected column, (new - old activation) times its W2 row, written out term by term
+    x, W1, b1, W2, b2 = _mlp_case(T=18, D=40, H=300, seed=8)
+    g = np.random.default_rng(13)
+    A = g.standard_normal((18, 300))
+    Y = g.standard_normal((18, 40))
+    idx = np.sort(np.stack([g.choice(300, 150, replace=False) for _ in range(3)]), axis=1).astype(np.int32)
+    A1, Y1 = O.mlp_delta(x, W1, b1, W2, idx, A, Y, Bt=8)
+    for b, r0, r1 in [(0, 0, 8), (1, 8, 16), (2, 16, 18)]:
+        a_new, _ = _mlp_brute(x[r0:r1], W1, b1, W2, b2, cols=idx[b].tolist())
+        for t in range(r1 - r0):
+            for n in range(40):
+                s = 0.0
+                for c in idx[b]:
+                    s += (a_new[t, c] - A[r0 + t, c]) * W2[c, n]
+                assert abs(Y1[r0 + t, n] - (Y[r0 + t, n] + s)) <= 1e-12
+            for c in idx[b]:
+                assert abs(A1[r0 + t, c] - a_new[t, c]) <= 1e-13 * max(1.0, abs(a_new[t, c]))
+    sel = np.zeros((18, 300), dtype=bool)
+    for b, r0, r1 in [(0, 0, 8), (1, 8, 16), (2, 16, 18)]:
+        sel[r0:r1, idx[b]] = True
+    np.testing.assert_array_equal(A1[~sel], A[~sel])
 
 
 def _consistent_cache(x_prev, W1, b1, W2, b2):
