@@ -134,3 +134,30 @@ def check_selection(idx, ref_scores, k, band):
         if k and k < n:
             assert ref_scores[r][mask].min() >= ref_scores[r][~mask].max() - band * scale, f"row {r}"
     return same
+
+
+def assert_is_topk_of(idx, scores, what: str):
+    """Each row of ``idx`` is the exact top-k of the same row of ``scores`` (fp32 values, compared as
+    numbers, so -0 equals +0), ties to the lower index, strictly ascending. A property check of a
+    result against its own input: every kept score is >= every dropped one, and where the k-th value
+    ties, the kept copies are the lowest-indexed ones."""
+    idx = np.asarray(idx)
+    scores = np.asarray(scores, dtype=np.float32)
+    rows, k = idx.shape
+    n = scores.shape[1]
+    assert scores.shape[0] == rows
+    if k == 0:
+        return
+    assert np.all(np.diff(idx, axis=1) > 0) if k > 1 else True, f"{what}: not strictly ascending"
+    assert idx.min() >= 0 and idx.max() < n, f"{what}: index out of range"
+    for r in range(rows):
+        kept = np.zeros(n, dtype=bool)
+        kept[idx[r]] = True
+        tau = scores[r][kept].min()
+        if k < n:
+            dropped = scores[r][~kept]
+            assert dropped.max() <= tau, f"{what}: row {r} drops a score above a kept one"
+            tie_dropped = np.flatnonzero(~kept & (scores[r] == tau))
+            tie_kept = np.flatnonzero(kept & (scores[r] == tau))
+            if tie_dropped.size:
+                assert tie_kept.max() < tie_dropped.min(), f"{what}: row {r} breaks a tie toward a higher index"

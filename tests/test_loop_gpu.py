@@ -9,14 +9,22 @@ cache bf16, output cache and attention partial fp32).
 
 A refresh's selection is a decision taken on float scores that each side
 computes on its own, so where scores nearly tie both selections are correct.
-At every refresh the test checks what is unique, that the GPU's selection is
-exactly the top-k of the GPU's own fp32 scores, and checks the scores
-themselves against the oracle's; then both chains continue from the GPU's
-selection (on the attention side the oracle rebuilds its complement cache for
-it). After a few sparse steps the two chains' bf16 activation caches can
-differ by one ulp in places, and a column score sums |a - A_cache|, a small
-difference of close values, so the score bound here is looser than on a fresh
-cache: max |err| <= 5e-2 * RMS of the scores.
+Nothing computed on the GPU enters the oracle chain. At every refresh the test
+checks what is unique: the GPU's selection is exactly the top-k of the GPU's
+own fp32 scores (a property check of the result against its input), its
+scores agree with the oracle's, and its selection is a valid top-k of the
+oracle's scores within a small band. Then:
+* MLP: the refresh rebuilds both caches densely, whatever the selection, so
+  the oracle's selection is uploaded into the GPU layer and both chains go on
+  from the same selection.
+* Attention: the complement cache depends on the selection, so each chain
+  keeps its own; the outputs of the sparse steps are compared on the
+  (head, query-block) tiles whose selections agree (at least 90% of them).
+After a few sparse steps the two chains' bf16 activation caches differ by one
+ulp in places (the fraction is measured and printed before the second
+refresh), and a column score sums |a - A_cache|, a small difference of close
+values, so the score bound after the first refresh is looser than on a fresh
+cache: max |err| <= 5e-2 * RMS of the scores (the measured ratio is printed).
 The gap to a fully dense fp64 run (the method's own approximation error) is
 printed for information.
 """
@@ -27,7 +35,8 @@ import pytest
 
 import oracle as O
 from dynamic_column_sparse_b200 import synth
-from helpers import assert_parity, dev_bf16, err_stats, f64_of_bf16, heads_first
+from helpers import (assert_is_topk_of, assert_parity, bits_of, check_selection, dev_bf16, err_stats, f64_of_bf16,
+                     heads_first, to_token_major)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,16 +45,20 @@ STEPS = 10
 SCORE_MAX_OF_RMS = 5e-2
 
 
-def check_refresh_selection(gpu_idx, gpu_scores, ref_scores, k, what):
-    """The GPU's selection is the exact top-k of its own scores, which agree with the oracle's."""
+def check_refresh_selection(gpu_idx, gpu_scores, ref_scores, k, what, bound=SCORE_MAX_OF_RMS):
+    """The GPU's selection is the exact top-k of its own scores, which agree with the oracle's;
+    returns a bool per row: the GPU's selection equals the oracle's."""
     rows = gpu_idx.shape[0]
-    np.testing.assert_array_equal(gpu_idx, O.topk_cols(gpu_scores.reshape(rows, -1), k), err_msg=what)
-    g = gpu_scores.reshape(rows, -1).astype(np.float64)
+    g = gpu_scores.reshape(rows, -1)
     r = ref_scores.reshape(rows, -1)
-    mx, rms, _ = err_stats(g, r)
-    print(f"{what}: score max|err|/rms {mx / rms:.4f}, rows as the oracle's "
-          f"{int(np.sum(np.all(gpu_idx == O.topk_cols(O.f32(r), k), axis=1)))} of {rows}")
-    assert mx <= SCORE_MAX_OF_RMS * rms, f"{what}: scores"
+    assert_is_topk_of(gpu_idx, g, what)
+    mx, rms, _ = err_stats(g.astype(np.float64), r)
+    same = np.all(gpu_idx == O.topk_cols(O.f32(r), k), axis=1)
+    check_selection(gpu_idx, r, k, band=2e-3 if bound < 1e-2 else 2 * bound)
+    print(f"{what}: score max|err|/rms {mx / rms:.4f} (bound {bound}), rows as the oracle's "
+          f"{int(same.sum())} of {rows}")
+    assert mx <= bound * rms, f"{what}: scores"
+    return same
 
 
 def drift_chain(first_bits, seed, tid, sigma, steps):
@@ -71,13 +84,23 @@ def run_mlp_loop(T, D, H, permille, seed=3):
     A = Y = idx = None
     worst = 0.0
     for s in range(STEPS):
-        out = f64_of_bf16(sched.run(layer, s, dev_bf16(xs[s])))
         x = O.bf16_decode(xs[s])
+        if sched.is_dense(s) and A is not None:
+            # one-ulp drift of the GPU's bf16 activation cache against the oracle chain's, before it is rebuilt
+            gpu_A = O.bf16_decode(to_token_major(bits_of(layer.a_cache), T))
+            ref_A = O.bf16_decode(O.bf16_round(A))
+            diff = np.abs(gpu_A - ref_A)
+            ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref_A), 2.0 ** -126))) - 7)
+            print(f"MLP activation cache before the step-{s} refresh: {np.mean(diff != 0):.2e} of entries differ, "
+                  f"by at most {float((diff / ulp).max()):.1f} bf16 ulp of the oracle's value "
+                  f"(max |diff| {float(diff.max()):.2e}, RMS of the cache {float(np.sqrt(np.mean(ref_A ** 2))):.2e})")
+        out = f64_of_bf16(sched.run(layer, s, dev_bf16(xs[s])))
         if sched.is_dense(s):
             r = O.mlp_refresh(x, W1, B1, W2, B2, A, 128, k, first_step=A is None)
-            A, Y = r["a"], r["y"]
-            idx = layer.idx.cpu().numpy()
-            check_refresh_selection(idx, layer.scores.cpu().numpy(), r["scores"], k, f"MLP refresh, step {s}")
+            A, Y, idx = r["a"], r["y"], r["idx"]
+            check_refresh_selection(layer.idx.cpu().numpy(), layer.scores.cpu().numpy(), r["scores"], k,
+                                    f"MLP refresh, step {s}", bound=5e-3 if s == 0 else SCORE_MAX_OF_RMS)
+            layer.idx.copy_(torch.from_numpy(idx).cuda())   # both chains go on from the oracle's selection
         else:
             A, Y = O.mlp_delta(x, W1, B1, W2, idx, A, Y, 128)
         ratio, _ = assert_parity(out, Y, f"MLP output, step {s}", bf16_out=True)
@@ -100,23 +123,25 @@ def run_attn_loop(T, h, permille, seed=4):
     sched = Schedule(DENSE_STEPS)
     scale = 1.0 / math.sqrt(128)
     kk = O.k_from_density(T, permille)
-    cache = None
+    cache = match = None
     for s in range(STEPS):
         out = heads_first(f64_of_bf16(sched.run(layer, s, *(dev_bf16(chains[n][s]) for n in ("q", "k", "v")))))
         q, k, v = (np.ascontiguousarray(O.bf16_decode(chains[n][s]).transpose(1, 0, 2)) for n in ("q", "k", "v"))
         if sched.is_dense(s):
             r = O.attn_refresh(q, k, v, scale, 128, kk)
-            idx = layer.idx.cpu().numpy()
-            nb = idx.shape[1]
-            check_refresh_selection(idx.reshape(h * nb, kk), layer.scores.cpu().numpy(), r["mass"], kk,
-                                    f"attention refresh, step {s}")
-            m_c, l_c, acc_c = (r["m_c"], r["l_c"], r["acc_c"]) if np.array_equal(idx, r["idx"]) else \
-                O.complement_partial(q, k, v, idx, scale, 128)
+            nb = r["idx"].shape[1]
+            same = check_refresh_selection(layer.idx.cpu().numpy().reshape(h * nb, kk), layer.scores.cpu().numpy(),
+                                           r["mass"], kk, f"attention refresh, step {s}", bound=5e-3)
+            assert same.mean() >= 0.9, f"step {s}: only {same.mean():.2f} of the selections as the oracle's"
+            # rows of the tiles whose selections agree; each chain keeps its own selection and complement
+            match = np.repeat(same.reshape(h, nb), 128, axis=1)[:, :T]
             f = lambda a: O.f32(a).astype(np.float64)  # the partial is stored as fp32
-            cache, ref = (idx, f(m_c), f(l_c), f(acc_c)), r["O"]
+            cache, ref = (r["idx"], f(r["m_c"]), f(r["l_c"]), f(r["acc_c"])), r["O"]
+            ratio, _ = assert_parity(out, ref, f"attention output, step {s}", bf16_out=True)
         else:
             ref = O.attn_delta(q, k, v, *cache, scale, 128)
-        ratio, _ = assert_parity(out, ref, f"attention output, step {s}", bf16_out=True)
+            ratio, _ = assert_parity(out[match], ref[match], f"attention output, step {s} (matching tiles)",
+                                     bf16_out=True)
         print(f"attn step {s}: max|err|/rms {ratio:.4f}")
     torch.cuda.synchronize()
 
