@@ -6,16 +6,22 @@
 // taken; a stable block-wide compaction in index order then writes the result.
 //
 // Rows of up to kStagedMaxN scores are staged in shared memory once and run a
-// three-pass radix select (11 + 11 + 10 bits) there. Longer rows take two
-// vectorised passes over global memory (two rows in flight per SM): a 12-bit
-// histogram finds the bucket holding the k-th key, then every element at or
-// above that bucket is copied (key and index, in index order) into shared
-// memory, each warp appending its own segment of the row to its own region;
-// the remaining 20 bits are resolved and the output compacted there. If one
-// warp's region overflows while the row's candidates still fit, the regions
-// are laid end to end after a counting pass. A row whose candidates do not
-// fit at all, or that is not 16-byte aligned, falls back to the general path
-// that re-reads the row from global memory for every radix pass.
+// three-pass radix select (11 + 11 + 10 bits) there. Longer rows (two in
+// flight per SM) first try a sampled threshold: every stride-th float4 of the
+// row is read, two radix passes find the top 22 bits of the r-th largest
+// sampled key, r set about three standard deviations above the sample's
+// expected share of the k largest, and one vectorised pass over the row copies
+// every key at or above that (key and index, in index order) into shared memory, each warp appending
+// its own segment of the row to its own region; the exact k-th key and the
+// output come from the candidates there. If the sample misjudged the row (too
+// few or too many candidates), a 12-bit histogram of the whole row finds the
+// bucket holding the k-th key and the keys in it or above become the
+// candidates. If one warp's region overflows while the row's candidates still
+// fit, the regions are laid end to end after a counting pass. A row whose
+// candidates do not fit at all, or that is not 16-byte aligned, falls back to
+// the general path that re-reads the row from global memory for every radix
+// pass. Histogram increments are aggregated per warp and bin, so scores that
+// crowd into a few bins do not serialise on one shared-memory atomic each.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -29,6 +35,7 @@ constexpr int kItems = 8;             // consecutive elements per thread in the 
 constexpr int kStagedMaxN = 40960;    // 160 KB of keys in shared memory
 constexpr int kLongBins = 4096;       // first digit of the long-row path: the top 12 key bits
 constexpr int kLongCap = 12288;       // long-row candidates held in shared memory (96 KB: two CTAs per SM)
+constexpr int kSampleMaxK = 9216;     // the sampled-threshold path serves k up to 3/4 of the candidate buffer
 
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -199,6 +206,18 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams p) {
   }
 }
 
+// One shared-memory increment of hist[bin] for every lane that has `active`
+// set, one atomic per distinct bin of the warp (scores that crowd into a few
+// bins would otherwise serialise on them). Warp-collective: every lane of the
+// warp must call it.
+__device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
+  const unsigned am = __ballot_sync(0xffffffffu, active);
+  if (active) {
+    const unsigned peers = __match_any_sync(am, bin);
+    if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+  }
+}
+
 // Long rows (see the file comment). Dynamic shared memory holds the candidate
 // keys and indices: kLongCap entries each, split into one region per warp.
 __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p) {
@@ -232,49 +251,18 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
     }
     const float4 *src4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
-    // pass 1: histogram of the top 12 bits of every key
-    for (int i = tid; i < kLongBins; i += kThreads) hist[i] = 0;
-    if (tid == 0) s_overflow = 0;
-    __syncthreads();
-    for (int i0 = tid; i0 < n4; i0 += kUnroll * kThreads) {
-      float4 v[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int i = i0 + u * kThreads;
-        v[u] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (i0 + u * kThreads < n4) {
-          atomicAdd(&hist[ordered_key(v[u].x) >> 20], 1u);
-          atomicAdd(&hist[ordered_key(v[u].y) >> 20], 1u);
-          atomicAdd(&hist[ordered_key(v[u].z) >> 20], 1u);
-          atomicAdd(&hist[ordered_key(v[u].w) >> 20], 1u);
-        }
-      }
-    }
-    for (int i = 4 * n4 + tid; i < n; i += kThreads) atomicAdd(&hist[ordered_key(__ldg(src + i)) >> 20], 1u);
-    __syncthreads();
-    select_digit(hist, kLongBins, k, warp_tot, s_digit, s_above);
-    const uint32_t b1 = s_digit;
-    const int kk1 = k - static_cast<int>(s_above);   // keys to take from bucket b1
-    const uint32_t n_cand = s_above + hist[b1];       // keys in bucket b1 or above
-    __syncthreads();
-    if (n_cand > static_cast<uint32_t>(kLongCap)) {
-      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
-      continue;
-    }
-    // pass 2: warp w takes float4 elements [w seg, (w+1) seg) (the last warp also
-    // the < 4 trailing scalars) and appends every key in bucket b1 or above,
-    // with its index, in index order, to its own region of the buffer
-    // (region w at s_base[w]). If a region overflows, every warp counts its
-    // candidates first, the regions are laid end to end, and the segments are
-    // read a second time.
+    // Warp w takes float4 elements [w seg, (w+1) seg) (the last warp also the
+    // < 4 trailing scalars) and appends every key >= lo, with its index, in
+    // index order, to its own region of the buffer (region w at s_base[w]). If a
+    // region overflows, every warp counts its candidates first, and if they fit
+    // the regions are laid end to end and the segments are read a second time.
+    // Returns false (block-uniform) if the candidates do not fit at all.
     const int seg = (n4 + kWarps - 1) / kWarps;
     const int f_lo = min(warp * seg, n4), f_hi = min(f_lo + seg, n4);
     // one pass over this warp's segment: counts (write false) or appends into
     // wkey / widx up to cap entries; returns the count, sets over past cap
-    auto scan_segment = [&](bool write, uint32_t *wkey, int32_t *widx, uint32_t cap, bool &over) -> uint32_t {
+    auto scan_segment = [&](uint32_t lo, bool write, uint32_t *wkey, int32_t *widx, uint32_t cap,
+                            bool &over) -> uint32_t {
       uint32_t wcount = 0;
       over = false;
       // this lane's flagged keys of one step (up to 4, elements base..base+3), in lane order
@@ -282,7 +270,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
         uint32_t flags = 0, cnt = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          if (c < nvalid && (key[c] >> 20) >= b1) {
+          if (c < nvalid && key[c] >= lo) {
             flags |= 1u << c;
             ++cnt;
           }
@@ -334,39 +322,40 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
       }
       return wcount;
     };
-    {
+    auto gather_candidates = [&](uint32_t lo) -> bool {
+      if (tid == 0) s_overflow = 0;
+      __syncthreads();
       bool over;
-      const uint32_t wc = scan_segment(true, ckey + warp * kRegion, cidx + warp * kRegion, kRegion, over);
+      uint32_t wc = scan_segment(lo, true, ckey + warp * kRegion, cidx + warp * kRegion, kRegion, over);
       if (lane == 0) {
         warp_tot[warp] = wc;
         if (over) s_overflow = 1;
       }
-    }
-    __syncthreads();
-    const bool contiguous = s_overflow != 0;
-    if (contiguous) {
-      bool over;
-      const uint32_t wc = scan_segment(false, nullptr, nullptr, 0, over);
-      if (lane == 0) warp_tot[warp] = wc;
       __syncthreads();
-    }
-    if (tid == 0) {
-      uint32_t acc = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        s_pref[w] = acc;
-        s_base[w] = contiguous ? acc : static_cast<uint32_t>(w * kRegion);
-        acc += static_cast<uint32_t>(warp_tot[w]);
+      const bool contiguous = s_overflow != 0;
+      if (contiguous) {
+        wc = scan_segment(lo, false, nullptr, nullptr, 0, over);
+        if (lane == 0) warp_tot[warp] = wc;
+        __syncthreads();
       }
-      s_pref[kWarps] = acc;
-    }
-    __syncthreads();
-    if (contiguous) {
-      // the counts add up to n_cand <= kLongCap, so the regions laid end to end fit
-      bool over;
-      scan_segment(true, ckey + s_base[warp], cidx + s_base[warp], static_cast<uint32_t>(kLongCap), over);
+      if (tid == 0) {
+        uint32_t acc = 0;
+        for (int w = 0; w < kWarps; ++w) {
+          s_pref[w] = acc;
+          s_base[w] = contiguous ? acc : static_cast<uint32_t>(w * kRegion);
+          acc += static_cast<uint32_t>(warp_tot[w]);
+        }
+        s_pref[kWarps] = acc;
+      }
       __syncthreads();
-    }
-    const int count = static_cast<int>(s_pref[kWarps]);
+      if (s_pref[kWarps] > static_cast<uint32_t>(kLongCap)) return false;
+      if (contiguous) {
+        // the counts add up to at most kLongCap, so the regions laid end to end fit
+        scan_segment(lo, true, ckey + s_base[warp], cidx + s_base[warp], static_cast<uint32_t>(kLongCap), over);
+        __syncthreads();
+      }
+      return true;
+    };
     // candidate L of the concatenated (index-ordered) list
     auto cand_at = [&](int L, uint32_t &key, int32_t &idx) {
       int w = 0;
@@ -377,20 +366,141 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
       key = ckey[j];
       idx = cidx[j];
     };
+    // radix passes over the first `count` keys of `keys` (or, with keys null,
+    // over the candidates): from (prefix, mask, kk), the digits of passes
+    // p0 .. p1 - 1 of (21: 11 bits, 10: 11 bits, 0: 10 bits)
+    auto radix_select = [&](const uint32_t *keys, int count, uint32_t &prefix, uint32_t &mask, int &kk, int p0,
+                            int p1) {
+#pragma unroll 1
+      for (int pass = p0; pass < p1; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nbins = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        for (int b0 = warp * 32; b0 < count; b0 += kThreads) {   // warp-uniform
+          const int L = b0 + lane;
+          uint32_t key = 0;
+          if (L < count) {
+            if (keys) {
+              key = keys[L];
+            } else {
+              int32_t unused;
+              cand_at(L, key, unused);
+            }
+          }
+          warp_hist_add(hist, (key >> shift) & static_cast<uint32_t>(nbins - 1), L < count && (key & mask) == prefix);
+        }
+        __syncthreads();
+        select_digit(hist, nbins, kk, warp_tot, s_digit, s_above);
+        prefix |= s_digit << shift;
+        mask |= static_cast<uint32_t>(nbins - 1) << shift;
+        kk -= static_cast<int>(s_above);
+        __syncthreads();
+      }
+    };
+    // stable compaction over the candidates in index order
+    auto compact_candidates = [&](uint32_t tau, int kk) {
+      const int count = static_cast<int>(s_pref[kWarps]);
+      uint32_t run_gt = 0, run_eq = 0;
+      const int tile = kThreads * kItems;
+      for (int base = 0; base < count; base += tile) {
+        const int first = base + tid * kItems;
+        uint32_t keys[kItems];
+        int32_t ids[kItems];
+#pragma unroll
+        for (int e = 0; e < kItems; ++e) {
+          keys[e] = 0u;
+          ids[e] = 0;
+          if (first + e < count) cand_at(first + e, keys[e], ids[e]);
+        }
+        compact_tile(keys, first, count, tau, kk, k, run_gt, run_eq, warp_tot,
+                     [&](uint32_t pos, int e) { dst[pos] = ids[e]; });
+      }
+      __syncthreads();
+    };
+
+    // Path 1: a threshold from a sample. Every stride-th float4 of the row is
+    // read and the r-th largest sampled key is taken as the lower bound of the
+    // candidates, r chosen so that about k + 3 standard deviations of the
+    // sample lie above the row's k-th key; then the row is read once.
+    bool done = false;
+    if (k <= kSampleMaxK && n4 >= 64) {
+      const int stride = max(16, (4 * n4 + kLongCap - 1) / kLongCap);
+      const int ns = min((n4 + stride - 1) / stride, kLongCap / 4);
+      const int m = 4 * ns;
+      for (int i = tid; i < ns; i += kThreads) {
+        const float4 v = __ldg(src4 + static_cast<size_t>(i) * stride);
+        ckey[4 * i] = ordered_key(v.x);
+        ckey[4 * i + 1] = ordered_key(v.y);
+        ckey[4 * i + 2] = ordered_key(v.z);
+        ckey[4 * i + 3] = ordered_key(v.w);
+      }
+      __syncthreads();
+      const float expect = static_cast<float>(k) * static_cast<float>(m) / static_cast<float>(n);
+      const int r = min(m, static_cast<int>(ceilf(expect + 3.f * sqrtf(expect))) + 8);
+      uint32_t prefix = 0, mask = 0;
+      int rr = r;
+      radix_select(ckey, m, prefix, mask, rr, 0, 2);
+      const uint32_t lo = prefix;   // the top 22 bits of the r-th largest sampled key (the rest zero)
+      if (gather_candidates(lo) && s_pref[kWarps] >= static_cast<uint32_t>(k)) {
+        uint32_t tau = 0, tmask = 0;
+        int kk = k;
+        radix_select(nullptr, static_cast<int>(s_pref[kWarps]), tau, tmask, kk, 0, 3);
+        compact_candidates(tau, kk);
+        done = true;
+      }
+    }
+    if (done) continue;
+
+    // Path 2: a 12-bit histogram of every key finds the bucket holding the
+    // k-th key; the keys in it or above are the candidates.
+    for (int i = tid; i < kLongBins; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = warp * 32; base < n4; base += kUnroll * kThreads) {   // warp-uniform
+      float4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int i = base + lane + u * kThreads;
+        v[u] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const bool valid = base + lane + u * kThreads < n4;
+        warp_hist_add(hist, ordered_key(v[u].x) >> 20, valid);
+        warp_hist_add(hist, ordered_key(v[u].y) >> 20, valid);
+        warp_hist_add(hist, ordered_key(v[u].z) >> 20, valid);
+        warp_hist_add(hist, ordered_key(v[u].w) >> 20, valid);
+      }
+    }
+    if (warp == 0) {
+      const int i = 4 * n4 + lane;
+      warp_hist_add(hist, i < n ? ordered_key(__ldg(src + i)) >> 20 : 0u, i < n);
+    }
+    __syncthreads();
+    select_digit(hist, kLongBins, k, warp_tot, s_digit, s_above);
+    const uint32_t b1 = s_digit;
+    const int kk1 = k - static_cast<int>(s_above);   // keys to take from bucket b1
+    const uint32_t n_cand = s_above + hist[b1];       // keys in bucket b1 or above
+    __syncthreads();
+    if (n_cand > static_cast<uint32_t>(kLongCap) || !gather_candidates(b1 << 20)) {
+      row_generic<false>(src, dst, n, k, nullptr, hist, warp_tot, s_digit, s_above);
+      continue;
+    }
     // the remaining 20 bits (10 + 10) among the candidates of bucket b1
     uint32_t prefix = b1 << 20, mask = 0xfff00000u;
     int kk = kk1;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
       const int shift = pass == 0 ? 10 : 0;
+      const int count = static_cast<int>(s_pref[kWarps]);
       for (int i = tid; i < 1024; i += kThreads) hist[i] = 0;
       __syncthreads();
-      for (int w = 0; w < kWarps; ++w) {
-        const int cw = static_cast<int>(s_pref[w + 1] - s_pref[w]);
-        for (int j = tid; j < cw; j += kThreads) {
-          const uint32_t key = ckey[s_base[w] + j];
-          if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
-        }
+      for (int b0 = warp * 32; b0 < count; b0 += kThreads) {   // warp-uniform
+        const int L = b0 + lane;
+        uint32_t key = 0;
+        int32_t unused;
+        if (L < count) cand_at(L, key, unused);
+        warp_hist_add(hist, (key >> shift) & 1023u, L < count && (key & mask) == prefix);
       }
       __syncthreads();
       select_digit(hist, 1024, kk, warp_tot, s_digit, s_above);
@@ -399,24 +509,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
       kk -= static_cast<int>(s_above);
       __syncthreads();
     }
-    const uint32_t tau = prefix;
-    // stable compaction over the candidates in index order
-    uint32_t run_gt = 0, run_eq = 0;
-    const int tile = kThreads * kItems;
-    for (int base = 0; base < count; base += tile) {
-      const int first = base + tid * kItems;
-      uint32_t keys[kItems];
-      int32_t ids[kItems];
-#pragma unroll
-      for (int e = 0; e < kItems; ++e) {
-        keys[e] = 0u;
-        ids[e] = 0;
-        if (first + e < count) cand_at(first + e, keys[e], ids[e]);
-      }
-      compact_tile(keys, first, count, tau, kk, k, run_gt, run_eq, warp_tot,
-                   [&](uint32_t pos, int e) { dst[pos] = ids[e]; });
-    }
-    __syncthreads();
+    compact_candidates(prefix, kk);
   }
 }
 

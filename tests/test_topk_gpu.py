@@ -97,3 +97,20 @@ def test_topk_long_rows_clustered_candidates(cm):
     s[2, 30000:34000] = hot[2]                            # and, on one row, in two such runs
     got = cm.topk_cols(dev_f32(s.astype(np.float32)), k).cpu().numpy()
     np.testing.assert_array_equal(got, O.topk_cols(s.astype(np.float32), k))
+
+
+def test_topk_long_rows_crowded_and_adversarial_samples(cm):
+    """Rows whose values crowd a few 12-bit key buckets, like attention-mass rows (all near
+    128 / T), and rows built against the sampled threshold of the long-row path: the largest
+    values only where the sample does not look (the threshold comes out too low: too many
+    candidates) or only where it looks (too high: too few)."""
+    n, k = 118800, 8316
+    z = synth.normal_f64(19, 1, 4 * n).reshape(4, n)
+    rows = [1e-3 * (1.0 + 0.1 * z[0]), 1e-3 * (1.0 + 0.01 * z[1])]
+    sampled = (np.arange(n) // 4) % 16 == 0              # float4 elements 0, 16, 32, ... are sampled
+    r = 1e-3 * (1.0 + 0.1 * np.abs(z[2])); r[~sampled] += 1.0; rows.append(r)
+    r = 1e-3 * (1.0 + 0.1 * np.abs(z[3])); r[sampled] += 1.0; rows.append(r)
+    s = np.stack(rows).astype(np.float32)
+    for kk in (k, 1, 9216, 9217):
+        got = cm.topk_cols(dev_f32(s), kk).cpu().numpy()
+        np.testing.assert_array_equal(got, O.topk_cols(s, kk), err_msg=f"k={kk}")
