@@ -545,7 +545,40 @@ def step_rows(Lx, w, reps, flush, torch):
     return out
 
 
-ROW_GROUPS = ("topk", "cols", "refresh", "dense", "sweep", "compact", "workloads", "cublas")
+ROW_GROUPS = ("topk", "cols", "refresh", "dense", "sweep", "compact", "workloads", "fp8", "cublas")
+
+
+def fp8_rows(Lx, w, reps, flush, torch, cm, peaks):
+    """The FP8 form of the sparse MLP step on layer Lx: x quantised per token (timed on its own), then
+    the gathered e4m3 GEMMs (chipmunk_mlp_delta_fp8). The weights are quantised once, outside the
+    timing; the deltas use a static scale that covers |delta| <= 0.5."""
+    T, D, H = w["T"], w["D"], w["H"]
+    w1t8, s1 = cm.quantize_e4m3_rows(Lx.w1t)
+    w2_8, s2 = cm.quantize_e4m3_rows(Lx.w2)
+    s_delta = float(s2.max().item()) * 0.5 / 448.0
+    g2 = (s2 / s_delta).float().contiguous()
+    x8 = torch.empty((T, D), dtype=torch.uint8, device=Lx.dev)
+    sx = torch.empty((T,), dtype=torch.float32, device=Lx.dev)
+    ws = torch.empty(cm.mlp_fp8_workspace_bytes(T, H, Lx.kc), dtype=torch.uint8, device=Lx.dev)
+    it = [0]
+
+    def quant():
+        cm.quantize_e4m3_rows(Lx.xs[it[0] % 2], x8, sx)
+
+    def step():
+        it[0] += 1
+        cm.mlp_delta_fp8(x8, sx, w1t8, s1, Lx.b1, w2_8, g2, s_delta, Lx.idx, Lx.a_cache, Lx.y_cache, Lx.out,
+                         workspace=ws)
+    quant()
+    step()
+    ms_q = time_events(quant, reps, flush, torch)
+    ms_s = time_events(step, reps, flush, torch)
+    flops = 4 * T * D * Lx.kc
+    fp8_peak = 2.0 * peaks["bf16_tflops"]   # the measured bf16 peak times the nominal fp8 / bf16 ratio
+    return {"T": T, "mlp_k": Lx.kc, "quantize_x_us": round(ms_q * 1e3, 1), "mlp_fp8_us": round(ms_s * 1e3, 1),
+            "tflops": round(flops / (ms_s * 1e-3) / 1e12, 1),
+            "frac_fp8_peak": round(flops / (ms_s * 1e-3) / 1e12 / fp8_peak, 4),
+            "peak_note": "fp8 peak = 2 x measured bf16 burst (nominal ratio)"}
 
 
 def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
@@ -573,6 +606,9 @@ def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
         rows["flux_2304x1280_step"] = step_rows(L2, w2, 5, flush, torch)
         del L2
         torch.cuda.empty_cache()
+    if "fp8" in groups:
+        rows["fp8_mlp_flux_1280x768"] = fp8_rows(LF, wf, 10, flush, torch, cm, peaks)
+        rows["fp8_mlp_hunyuan"] = fp8_rows(L, w, 3, flush, torch, cm, peaks)
     if "topk" in groups:
         topk_rows(LF, wf, rows, gbs, flush, torch, cm)
     if "cols" in groups:

@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(_HERE, "libchipmunk.so")
 
 OK = 0
 ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGNMENT, ERR_CUDA, ERR_DEVICE, ERR_UNSUPPORTED, ERR_WORKSPACE = 1, 2, 3, 4, 5, 6, 7
-OP_TOPK, OP_MLP_DELTA, OP_ATTN_DELTA, OP_REFRESH = 0, 1, 2, 3
+OP_TOPK, OP_MLP_DELTA, OP_ATTN_DELTA, OP_REFRESH, OP_MLP_DELTA_FP8 = 0, 1, 2, 3, 4
 REFRESH_MLP, REFRESH_ATTN = 0, 1
 
 EXPORTS = (
@@ -37,7 +37,7 @@ EXPORTS = (
     "chipmunk_attn_delta", "chipmunk_dense_refresh",
     "chipmunk_gather_cols", "chipmunk_scatter_cols", "chipmunk_workspace_bytes", "chipmunk_status_string",
     "chipmunk_last_error", "chipmunk_read_device_status", "chipmunk_version", "chipmunk_mlp_delta_noalloc",
-    "chipmunk_selftest_bounded_wait",
+    "chipmunk_selftest_bounded_wait", "chipmunk_mlp_delta_fp8", "chipmunk_quantize_e4m3_rows",
 )
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -55,6 +55,16 @@ class MlpArgs(ctypes.Structure):
         ("x", ctypes.c_void_p), ("w1t", ctypes.c_void_p), ("b1", ctypes.c_void_p),
         ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("idx", ctypes.c_void_p),
         ("a_cache", ctypes.c_void_p), ("y_cache", ctypes.c_void_p), ("out", ctypes.c_void_p),
+    ]
+
+
+class MlpFp8Args(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int64), ("D", ctypes.c_int64), ("H", ctypes.c_int64),
+        ("Bt", ctypes.c_int32), ("k", ctypes.c_int32),
+        ("x8", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("w1t8", ctypes.c_void_p), ("s1", ctypes.c_void_p),
+        ("b1", ctypes.c_void_p), ("w2_8", ctypes.c_void_p), ("g2", ctypes.c_void_p), ("s_delta", ctypes.c_float),
+        ("idx", ctypes.c_void_p), ("a_cache", ctypes.c_void_p), ("y_cache", ctypes.c_void_p), ("out", ctypes.c_void_p),
     ]
 
 
@@ -102,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "chipmunk_read_device_status": [ctypes.POINTER(i32), vp],
             "chipmunk_mlp_delta_noalloc": [ctypes.POINTER(MlpArgs), vp],
             "chipmunk_selftest_bounded_wait": [vp],
+            "chipmunk_mlp_delta_fp8": [ctypes.POINTER(MlpFp8Args), vp, sz, vp],
+            "chipmunk_quantize_e4m3_rows": [vp, i64, i64, vp, vp, vp],
         }
         for name, argtypes in sig.items():
             fn = getattr(lib, name)
@@ -248,6 +260,73 @@ def mlp_refresh(x, w1t, b1, w2, b2, a_cache, y_cache, idx, scores, out=None, Bt=
     _need(scores, "scores", torch.float32, (a_cache.shape[0], w1t.shape[0]))
     r = RefreshArgs(REFRESH_MLP, 1 if first_step else 0, a, AttnArgs(), scores.data_ptr())
     _check(lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ FP8 MLP step
+
+def _need_codes(t, name, shape):
+    """e4m3 codes: torch.uint8 or torch.float8_e4m3fn storage."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+        raise TypeError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn), got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def quantize_e4m3_rows(x, codes=None, scales=None, stream=None):
+    """Rows of bf16 x [R][C] to e4m3 codes [R][C] (uint8) and per-row fp32 scales [R]: x ~ scale * code."""
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    R, C = x.shape
+    if codes is None:
+        codes = torch.empty((R, C), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((R,), dtype=torch.float32, device=x.device)
+    _need_codes(codes, "codes", (R, C))
+    _need(scales, "scales", torch.float32, (R,))
+    _check(lib.chipmunk_quantize_e4m3_rows(_ptr(x), R, C, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def mlp_fp8_workspace_bytes(T: int, H: int, k: int) -> int:
+    return workspace_bytes(OP_MLP_DELTA_FP8, MlpFp8Args(T, 256, H, 128, k))
+
+
+def mlp_delta_fp8(x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, a_cache, y_cache, out=None, workspace=None,
+                  stream=None):
+    """FP8 form of the sparse MLP step (chipmunk_mlp_delta_fp8): e4m3 operands with per-token (sx),
+    per-hidden-unit (s1) scales, deltas rounded to e4m3 after multiplying by g2 = s2 / s_delta."""
+    lib = load_library()
+    T, D = x8.shape
+    H = w1t8.shape[0]
+    nb = (T + 127) // 128
+    k = idx.shape[1]
+    _need_codes(x8, "x8", (T, D))
+    _need(sx, "sx", torch.float32, (T,))
+    _need_codes(w1t8, "w1t8", (H, D))
+    _need(s1, "s1", torch.float32, (H,))
+    _need(b1, "b1", torch.bfloat16, (H,))
+    _need_codes(w2_8, "w2_8", (H, D))
+    _need(g2, "g2", torch.float32, (H,))
+    _need(idx, "idx", torch.int32, (nb, k))
+    _need(a_cache, "a_cache", torch.bfloat16, (nb, H, 128))
+    _need(y_cache, "y_cache", torch.float32, (T, D))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (T, D))
+    a = MlpFp8Args(T, D, H, 128, k, x8.data_ptr(), sx.data_ptr(), w1t8.data_ptr(), s1.data_ptr(), b1.data_ptr(),
+                   w2_8.data_ptr(), g2.data_ptr(), float(s_delta), idx.data_ptr(), a_cache.data_ptr(),
+                   y_cache.data_ptr(), 0 if out is None else out.data_ptr())
+    need = workspace_bytes(OP_MLP_DELTA_FP8, a)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x8.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.chipmunk_mlp_delta_fp8(ctypes.byref(a), _ptr(workspace), ws_bytes, _stream(stream)))
     return out
 
 

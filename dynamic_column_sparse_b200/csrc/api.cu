@@ -82,9 +82,10 @@ chipmunk_status device_setup(int **status_out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// bf16 tensor map of rank 2 or 3 with 128-byte swizzle. dims/box innermost first.
+// Tensor map of rank 2 or 3 with 128-byte swizzle (bf16 elements, or bytes when
+// `bytes` is set). dims/box innermost first.
 chipmunk_status make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
-                         const uint32_t *box, const char *what) {
+                         const uint32_t *box, const char *what, bool bytes = false) {
   cuuint64_t gd[3], gs[2];
   cuuint32_t bx[3], es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) {
@@ -92,7 +93,8 @@ chipmunk_status make_map(CUtensorMap *m, const void *base, int rank, const uint6
     bx[i] = box[i];
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
+  CUresult r = g_encode(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                        const_cast<void *>(base), gd, gs, bx, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CHIPMUNK_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, int(r));
@@ -233,6 +235,30 @@ chipmunk_status mlp_down_impl(const chipmunk_mlp_args *a, void *ws, int *status,
   return CHIPMUNK_OK;
 }
 
+chipmunk_status check_mlp_fp8(const chipmunk_mlp_fp8_args *a) {
+  if (a == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "args is NULL");
+  if (a->T < 1 || a->T > (int64_t(1) << 30)) return fail(CHIPMUNK_ERR_SHAPE, "T=%lld out of range", (long long)a->T);
+  if (a->D < 256 || a->D > 16384 || a->D % 256 != 0)
+    return fail(CHIPMUNK_ERR_SHAPE, "D=%lld must be a multiple of 256 in [256, 16384] for the FP8 step", (long long)a->D);
+  if (a->H < 1 || a->H > (int64_t(1) << 24)) return fail(CHIPMUNK_ERR_SHAPE, "H=%lld out of range", (long long)a->H);
+  if (a->Bt != 128) return fail(CHIPMUNK_ERR_SHAPE, "Bt=%d: the FP8 step is built for 128", a->Bt);
+  if (a->k < 0 || a->k > a->H) return fail(CHIPMUNK_ERR_INVALID_ARG, "k=%d outside [0, H=%lld]", a->k, (long long)a->H);
+  if (!(a->s_delta > 0.f) || !std::isfinite(a->s_delta)) return fail(CHIPMUNK_ERR_INVALID_ARG, "s_delta must be > 0");
+  const void *req[] = {a->x8, a->sx, a->w1t8, a->s1, a->b1, a->w2_8, a->g2, a->a_cache, a->y_cache, a->idx};
+  const char *names[] = {"x8", "sx", "w1t8", "s1", "b1", "w2_8", "g2", "a_cache", "y_cache", "idx"};
+  for (int i = 0; i < 10; ++i) {
+    if (req[i] == nullptr && !(i == 9 && a->k == 0)) return fail(CHIPMUNK_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (req[i] != nullptr && !aligned16(req[i])) return fail(CHIPMUNK_ERR_ALIGNMENT, "%s is not 16-byte aligned", names[i]);
+  }
+  if (a->out != nullptr && !aligned16(a->out)) return fail(CHIPMUNK_ERR_ALIGNMENT, "out is not 16-byte aligned");
+  return CHIPMUNK_OK;
+}
+
+size_t mlp_delta_fp8_ws(const chipmunk_mlp_fp8_args *a) {
+  if (a->k <= 0) return 0;
+  return size_t(ceil_div(a->T, 128)) * size_t(ceil_div(a->k, 128) * 128) * 128;
+}
+
 }  // namespace
 
 namespace cm {
@@ -282,6 +308,8 @@ size_t chipmunk_workspace_bytes(int32_t op, const void *args) {
   switch (op) {
     case CHIPMUNK_OP_MLP_DELTA:
       return args ? mlp_delta_ws(static_cast<const chipmunk_mlp_args *>(args)) : 0;
+    case CHIPMUNK_OP_MLP_DELTA_FP8:
+      return args ? mlp_delta_fp8_ws(static_cast<const chipmunk_mlp_fp8_args *>(args)) : 0;
     case CHIPMUNK_OP_REFRESH: {
       if (!args) return 0;
       const chipmunk_refresh_args *r = static_cast<const chipmunk_refresh_args *>(args);
@@ -326,6 +354,61 @@ chipmunk_status chipmunk_mlp_delta_down(const chipmunk_mlp_args *a, void *ws, si
   int *status = nullptr;
   CM_CHECK(mlp_delta_prologue(a, ws, ws_bytes, &status));
   return mlp_down_impl(a, ws, status, static_cast<cudaStream_t>(stream));
+}
+
+chipmunk_status chipmunk_mlp_delta_fp8(const chipmunk_mlp_fp8_args *a, void *ws, size_t ws_bytes,
+                                       chipmunk_stream stream) {
+  CM_CHECK(check_mlp_fp8(a));
+  const size_t need = mlp_delta_fp8_ws(a);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(CHIPMUNK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if (need > 0 && !aligned16(ws)) return fail(CHIPMUNK_ERR_ALIGNMENT, "ws is not 16-byte aligned");
+  int *status = nullptr;
+  CM_CHECK(device_setup(&status));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nb = ceil_div(a->T, 128);
+  const int64_t nchunks = ceil_div(a->k, 128);
+  const int64_t k_pad = nchunks * 128;
+  if (a->k > 0) {
+    CUtensorMap tm_x;
+    {
+      const uint64_t dims[2] = {uint64_t(a->D), uint64_t(a->T)};
+      const uint64_t strides[1] = {uint64_t(a->D)};
+      const uint32_t box[2] = {128, 128};
+      CM_CHECK(make_map(&tm_x, a->x8, 2, dims, strides, box, "x8", true));
+    }
+    cm::MlpUpParams up{int(a->T), int(a->D), int(a->H), a->k, 128, int(nb), int(nchunks), int(k_pad), cm::kUpDelta,
+                       static_cast<const uint16_t *>(a->w1t8), a->idx, static_cast<const uint16_t *>(a->b1),
+                       static_cast<uint16_t *>(a->a_cache), static_cast<uint16_t *>(ws), nullptr, status,
+                       a->sx, a->s1, a->g2};
+    CM_CUDA(cm::launch_mlp_up_fp8(up, tm_x, s), "FP8 MLP up-projection launch");
+  }
+  cm::MlpDownParams dp{int(a->T), int(a->D), 128, int(nb), int(k_pad), a->k, int(a->D / 256), 256,
+                       cm::kDownAccumulate, static_cast<const uint16_t *>(a->w2_8), int(a->H), a->idx, nullptr,
+                       a->y_cache, static_cast<uint16_t *>(a->out), status, a->s_delta};
+  CUtensorMap tm_d;
+  if (a->k > 0) {
+    const uint64_t dims[3] = {128, uint64_t(k_pad), uint64_t(nb)};
+    const uint64_t strides[2] = {128, uint64_t(k_pad) * 128};
+    const uint32_t box[3] = {128, 128, 1};
+    CM_CHECK(make_map(&tm_d, ws, 3, dims, strides, box, "delta codes", true));
+  }
+  CM_CUDA(cm::launch_mlp_down_fp8(dp, tm_d, s), "FP8 MLP down-projection launch");
+  return CHIPMUNK_OK;
+}
+
+chipmunk_status chipmunk_quantize_e4m3_rows(const void *x, int64_t rows, int64_t cols, void *codes, float *scales,
+                                            chipmunk_stream stream) {
+  if (rows < 0 || cols < 16 || cols % 16 != 0) return fail(CHIPMUNK_ERR_SHAPE, "rows/cols out of range (cols a multiple of 16)");
+  if (rows == 0) return CHIPMUNK_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(x) || !aligned16(codes)) return fail(CHIPMUNK_ERR_ALIGNMENT, "x or codes not 16-byte aligned");
+  int *status = nullptr;
+  CM_CHECK(device_setup(&status));
+  CM_CUDA(cm::launch_quantize_e4m3_rows(static_cast<const uint16_t *>(x), rows, cols, static_cast<uint8_t *>(codes),
+                                        scales, status, static_cast<cudaStream_t>(stream)),
+          "quantize launch");
+  return CHIPMUNK_OK;
 }
 
 chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, void *ws, size_t ws_bytes, chipmunk_stream stream) {

@@ -35,16 +35,22 @@ enum MlpUpMode : int { kUpDelta = 0, kUpRefresh = 1, kUpRefreshFirst = 2 };
 // epilogue. One CTA per (token block, chunk of 128 selected columns).
 struct MlpUpParams {
   int T, D, H, k, Bt, nb, nchunks, k_pad, mode;
-  const uint16_t *w1t;    // [H][D] (rows gathered on a sparse step)
+  const uint16_t *w1t;    // [H][D] (rows gathered on a sparse step); e4m3 codes [H][D] in the FP8 step
   const int32_t *idx;     // [nb][k] (sparse step)
   const uint16_t *b1;     // [H]
   uint16_t *a_cache;      // [nb][H][Bt]
-  uint16_t *delta;        // [nb][k_pad][Bt] (sparse step)
+  uint16_t *delta;        // [nb][k_pad][Bt] (sparse step); e4m3 codes in the FP8 step
   float *scores;          // [nb][H] (refresh)
   int *status;
+  // FP8 step only: x ~ sx[t] * x8[t][:], W1^T ~ s1[c] * w1t8[c][:], the delta
+  // of column c is multiplied by g2[c] before it is rounded to e4m3
+  const float *sx, *s1, *g2;
 };
 // tm_w1t: tile map over W1^T [H][D] (box 64 x 128), read on a refresh only.
 cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s);
+// The sparse step with e4m3 operands (Bt = 128): tm_x is a byte map over the
+// codes x8 [T][D] (box 128 x 128); the deltas are written as e4m3 codes.
+cudaError_t launch_mlp_up_fp8(const MlpUpParams &p, const CUtensorMap &tm_x, cudaStream_t s);
 
 enum MlpDownMode : int { kDownAccumulate = 0, kDownOverwrite = 1 };
 
@@ -53,17 +59,27 @@ enum MlpDownMode : int { kDownAccumulate = 0, kDownOverwrite = 1 };
 // cache (refresh, all rows). One CTA per (token block, slice of BN columns).
 struct MlpDownParams {
   int T, D, Bt, nb, krows, k, n_slices, bn, mode;
-  const uint16_t *w2;     // [H][D] (rows gathered on a sparse step)
+  const uint16_t *w2;     // [H][D] (rows gathered on a sparse step); e4m3 codes [H][D] in the FP8 step
   int H;
   const int32_t *idx;     // [nb][k] (sparse step)
   const uint16_t *b2;     // [D] (refresh)
   float *y_cache;         // [T][D]
   uint16_t *out;          // [T][D] or nullptr
   int *status;
+  float s_delta;          // FP8 step only: the scale of the delta codes
 };
 // tm_a: 3-D map over A [nb][rows][Bt]; tm_w2: tile map over W2 [H][D] (box 64 x 64), read on a refresh only.
 cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
                             cudaStream_t s);
+// The sparse step with e4m3 operands (Bt = 128, D a multiple of 256): tm_a is
+// a byte map over the delta codes [nb][k_pad][128] (box 128 x 128 x 1).
+cudaError_t launch_mlp_down_fp8(const MlpDownParams &p, const CUtensorMap &tm_a, cudaStream_t s);
+
+// ------------------------------------------------------------------ FP8 quantisation
+
+// codes[r][:] = e4m3(x[r][:] / scales[r]), scales[r] = max |x[r][:]| / 448 (1 for an all-zero row).
+cudaError_t launch_quantize_e4m3_rows(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *codes, float *scales,
+                                      int *status, cudaStream_t s);
 
 // ------------------------------------------------------------------ attention
 

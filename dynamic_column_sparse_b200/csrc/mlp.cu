@@ -30,6 +30,8 @@
 // gathered stage and hands the stage on through a second barrier, because the
 // fence stalls whichever warp executes it and the MMA warp is mlp_up's
 // critical path (mlp_down's MMA warp takes it itself at no measurable cost).
+#include <cuda_fp8.h>
+
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -83,18 +85,27 @@ struct UpCfg : Roles<4, 4> {
 // accumulators alternate between tiles, so the epilogue of one tile overlaps
 // the main loop of the next; ring stages and parities follow one running
 // k-step counter across tiles.
-template <int BT, bool DENSE>
+//
+// F8: the FP8 form of the sparse step. x and W1^T arrive as e4m3 codes; a
+// stage still holds 128-byte rows, now of 128 K elements, and the tensor core
+// runs kind::f8f6f4 (K = 32 per instruction). The epilogue scales the fp32
+// accumulator by s1[c] * sx[t] before the bias, and writes each delta as the
+// e4m3 code of delta * g2[c] (the down-projection's operand).
+template <int BT, bool DENSE, bool F8 = false>
 __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
     mlp_up_kernel(const __grid_constant__ CUtensorMap tm_w1t, const __grid_constant__ CUtensorMap tm_x,
                   const MlpUpParams p) {
   using C = UpCfg<BT>;
+  static_assert(!F8 || (BT == 128 && !DENSE), "the FP8 step runs the sparse form with 128-token blocks");
   constexpr int SA = C::kStagesA, SB = C::kStagesB;
   constexpr int kProducers = C::kProducers, kMmaWarp = C::kMmaWarp, kTmaWarp = C::kTmaWarp;
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
   constexpr int kParts = C::kEpiWarps / 4;  // epilogue warps per TMEM lane quadrant
   constexpr int kHalf = BT / kParts;         // accumulator columns (tokens) of one epilogue warp
   constexpr int kRowIters = 1024 / kProducers;  // gathered rows of a stage per producer thread
-  constexpr uint32_t kIdesc = idesc_bf16(128, BT, false, false);
+  constexpr int kEs = F8 ? 1 : 2;               // bytes per operand element
+  constexpr int kKStage = 128 / kEs;            // K elements per stage (one 128-byte swizzle row)
+  constexpr uint32_t kIdesc = F8 ? idesc_e4m3(128, BT, false, false) : idesc_bf16(128, BT, false, false);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
@@ -118,7 +129,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
   const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
                            ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                            : 0;
-  const int nk = p.D / kBK;
+  const int nk = p.D / kKStage;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -175,8 +186,9 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       const uint32_t a_base = smem_u32(sA);
       int kg = 0;
       bool ok = true;
+      const uint8_t *w1b = reinterpret_cast<const uint8_t *>(p.w1t);
       for (int tl = 0; tl < my_tiles && ok; ++tl) {
-        const uint16_t *src_row[kRowIters];
+        const uint8_t *src_row[kRowIters];   // this thread's 16-byte piece of each gathered row
 #pragma unroll
         for (int i = 0; i < kRowIters; ++i) {
           int c = nxt[i];
@@ -184,7 +196,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
             atomicCAS(p.status, kDevOk, kDevBadIndex);
             c = 0;
           }
-          src_row[i] = p.w1t + static_cast<size_t>(c) * p.D + (pt & 7) * 8;
+          src_row[i] = w1b + static_cast<size_t>(c) * p.D * kEs + (pt & 7) * 16;
         }
         load_rows(tl + 1, nxt);
         for (int kb = 0; kb < nk; ++kb, ++kg) {
@@ -195,7 +207,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
           }
           const uint32_t stage = a_base + s * C::kABytes;
 #pragma unroll
-          for (int i = 0; i < kRowIters; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * kBK);
+          for (int i = 0; i < kRowIters; ++i) cp_async_16(stage + dst_off[i], src_row[i] + kb * 128);
           cp_async_arrive_noinc(&a_full[s]);
         }
       }
@@ -226,7 +238,7 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&b_full[s], C::kBBytes);
-          tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kBK, b * BT);
+          tma_load_2d(sB + s * C::kBBytes, &tm_x, &b_full[s], kb * kKStage, b * BT);
         }
         __syncwarp();
         if (!DENSE && kg >= 1) {
@@ -270,10 +282,13 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
           const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
           const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {   // 32 bytes of K per instruction
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+            if (F8)
+              umma_e4m3(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+            else
+              umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
           }
           umma_commit(&a_empty[sa]);
           umma_commit(&b_empty[sb]);
@@ -319,6 +334,8 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
         c = min(j, p.H - 1);
       }
       const float bias = bf16_bits_to_f32(__ldg(p.b1 + c));
+      const float s1c = F8 ? __ldg(p.s1 + c) : 1.f;   // FP8: scale of the column's W1^T row
+      const float g2c = F8 ? __ldg(p.g2 + c) : 0.f;   // FP8: factor of the column's delta before rounding
       const int nvalid = min(BT, p.T - b * BT);
       const bool need_old = valid_j && !(first && !sparse);
       // the columns whose runs this lane moves: 8 i + cq, i = 0..3
@@ -358,6 +375,9 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
           mbar_arrive(&acc_empty[ab]);  // the accumulator can take the next-but-one tile
         }
         const uint16_t *old = reinterpret_cast<const uint16_t *>(oldw);
+        // FP8: the scale of token 32 tq + lane, handed to every lane by shuffles
+        const int t_lane = th * kHalf + tq * 32 + lane;
+        const float sx_lane = F8 && t_lane < nvalid ? __ldg(p.sx + static_cast<size_t>(b) * BT + t_lane) : 0.f;
         uint32_t na[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -365,7 +385,9 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = th * kHalf + tq * 32 + i + u;
-            const float a = gelu_tanh(acc[i + u] + bias);
+            float pre_act = acc[i + u] + bias;
+            if (F8) pre_act = fmaf(acc[i + u], s1c * __shfl_sync(0xffffffffu, sx_lane, i + u), bias);
+            const float a = gelu_tanh(pre_act);
             const bool tok = t < nvalid;
             nab[u] = tok ? f32_to_bf16_bits(a) : old[i + u];
             if (!sparse) score += tok ? fabsf(first ? a : a - bf16_bits_to_f32(old[i + u])) : 0.f;
@@ -388,7 +410,29 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
           for (int i = 0; i < 4; ++i)
             pre[i] = (old_mask >> i) & 1 ? *reinterpret_cast<const uint4 *>(arun(i) + (tq + 1) * 32) : make_uint4(0, 0, 0, 0);
         }
-        if (sparse) {
+        if (F8) {
+          // the e4m3 code of (bf16(new) - old) * g2[c] for real tokens of a selected
+          // column, else 0; this column's 32 codes go straight out as two 16-byte pieces
+          const uint16_t *nw = reinterpret_cast<const uint16_t *>(na);
+          uint32_t cw[8];
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * w + e;
+              const bool tok = th * kHalf + tq * 32 + i < nvalid;
+              const float d = (bf16_bits_to_f32(nw[i]) - bf16_bits_to_f32(old[i])) * g2c;
+              const uint32_t code = (valid_j && tok) ? static_cast<uint32_t>(__nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3)) : 0u;
+              word |= code << (8 * e);
+            }
+            cw[w] = word;
+          }
+          uint8_t *drow = reinterpret_cast<uint8_t *>(p.delta) +
+                          (static_cast<size_t>(b) * p.k_pad + chunk * 128 + r) * BT + th * kHalf + tq * 32;
+          reinterpret_cast<uint4 *>(drow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          reinterpret_cast<uint4 *>(drow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        } else if (sparse) {
           // delta = bf16(new) - old for real tokens of a selected column, else 0
           const uint16_t *nw = reinterpret_cast<const uint16_t *>(na);
           uint32_t dl[16];
@@ -815,18 +859,30 @@ struct DownCfg : Roles<8, 4> {   // eight gathering warps: the W2 stream is boun
 // accumulators alternate between tiles so the epilogue of one tile overlaps
 // the main loop of the next. Ring stages and their parities follow one
 // running k-step counter across tiles.
-template <int BT, int BN, bool DENSE>
+//
+// F8: the FP8 form of the sparse step. The delta codes and the gathered W2
+// rows are e4m3: a stage holds 128 K-rows (selected columns) of 128-byte
+// rows, the delta tile (128 tokens) arrives by one TMA load, the W2 row
+// segments (BN bytes) form BN / 128 slabs of 128 columns, the tensor core runs
+// kind::f8f6f4 (K = 32 per instruction) and the epilogue scales the result by
+// the deltas' scale before adding it to the output cache.
+template <int BT, int BN, bool DENSE, bool F8 = false>
 __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm)
     mlp_down_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w2,
                     const MlpDownParams p) {
   using C = DownCfg<BN>;
+  static_assert(!F8 || (BT == 128 && BN == 256 && !DENSE), "the FP8 step runs the sparse form, 128 x 256 tiles");
   constexpr int SA = C::kStagesA, SB = C::kStagesB;
   constexpr int kProducers = C::kProducers, kMmaWarp = C::kMmaWarp, kTmaWarp = C::kTmaWarp, kThreads = C::kThreads;
-  constexpr int kRowsPerWarp = kBK / C::kProdWarps;   // gathered W2 rows of a stage per producer warp
-  constexpr uint32_t kIdesc = idesc_bf16(128, BN, true, true);
-  constexpr uint32_t kATx = (BT / 64) * 8192;
-  constexpr int kChunksPerRow = BN / 8;               // 16-byte chunks of one gathered W2 row segment
+  constexpr int kEs = F8 ? 1 : 2;                     // bytes per operand element
+  constexpr int kKStage = 128 / kEs;                  // K rows (selected columns) per stage
+  constexpr int kRowsPerWarp = kKStage / C::kProdWarps;   // gathered W2 rows of a stage per producer warp
+  constexpr uint32_t kIdesc = F8 ? idesc_e4m3(128, BN, true, true) : idesc_bf16(128, BN, true, true);
+  constexpr uint32_t kATx = F8 ? 16384 : (BT / 64) * 8192;
+  constexpr int kChunksPerRow = BN * kEs / 16;        // 16-byte chunks of one gathered W2 row segment
   constexpr int kRowsPerInstr = 32 / kChunksPerRow;   // rows one warp instruction covers
+  constexpr uint32_t kSlabBytes = kKStage * 128;      // one 128-byte-wide column slab of a B stage
+  constexpr uint32_t kKStep = (F8 ? 32 : 16) * 128;   // bytes of the 128-byte K rows one MMA consumes
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align_up<1024>(smem_raw);
   uint8_t *sA = smem;
@@ -844,7 +900,7 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
   if (*(volatile int *)p.status != kDevOk) return;
   const int ntiles = p.nb * p.n_slices;
   const int kext = DENSE ? p.krows : p.k;
-  const int nk = (kext + kBK - 1) / kBK;
+  const int nk = (kext + kKStage - 1) / kKStage;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -905,7 +961,7 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
       auto load_idx = [&]() -> int {
         int c = 0;
         if (lane < kRowsPerWarp && ltile < ntiles)
-          c = __ldg(p.idx + static_cast<size_t>(ltile % p.nb) * p.k + min(lkb * kBK + pw * kRowsPerWarp + lane, p.k - 1));
+          c = __ldg(p.idx + static_cast<size_t>(ltile % p.nb) * p.k + min(lkb * kKStage + pw * kRowsPerWarp + lane, p.k - 1));
         if (++lkb == nk) {
           lkb = 0;
           ltile += gridDim.x;
@@ -928,8 +984,8 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
           const int r = pw * kRowsPerWarp + rr;      // row of the stage
           const int cr = __shfl_sync(0xffffffffu, c, rr);
           const int slab = csub >> 3, cc = csub & 7;
-          cp_async_16(stage + slab * 8192 + sw128_offset(r, cc),
-                      p.w2 + static_cast<size_t>(cr) * p.D + n0 + csub * 8);
+          cp_async_16(stage + slab * kSlabBytes + sw128_offset(r, cc),
+                      reinterpret_cast<const uint8_t *>(p.w2) + (static_cast<size_t>(cr) * p.D + n0) * kEs + csub * 16);
         }
         cp_async_arrive_noinc(&b_full[s]);
         if (++kb == nk) {
@@ -977,9 +1033,13 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&a_full[s], kATx);
+          if (F8) {
+            tma_load_3d(sA + s * C::kABytes, &tm_a, &a_full[s], 0, kb * kKStage, b);
+          } else {
 #pragma unroll
-          for (int mt = 0; mt < BT / 64; ++mt)
-            tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &a_full[s], mt * 64, kb * kBK, b);
+            for (int mt = 0; mt < BT / 64; ++mt)
+              tma_load_3d(sA + s * C::kABytes + mt * 8192, &tm_a, &a_full[s], mt * 64, kb * kBK, b);
+          }
         }
         __syncwarp();
       }
@@ -1005,10 +1065,15 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
           const uint32_t a0 = smem_u32(sA + sa * C::kABytes);
           const uint32_t b0 = smem_u32(sB + sb * C::kBBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a0 + kk * 2048, 8192, 1024);
-            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, 8192, 1024);
-            umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            // MN-major: A atoms of 128 bytes of tokens (two 64-token atoms 8 KB apart for bf16, one
+            // 128-token atom for e4m3), B slabs kSlabBytes apart, 8-row groups 1 KB apart
+            const uint64_t ad = sdesc_sw128(a0 + kk * kKStep, 8192, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * kKStep, kSlabBytes, 1024);
+            if (F8)
+              umma_e4m3(tacc, ad, bd, kIdesc, (kb | kk) != 0);
+            else
+              umma_bf16(tacc, ad, bd, kIdesc, (kb | kk) != 0);
           }
           umma_commit(&a_empty[sa]);
           umma_commit(&b_empty[sb]);
@@ -1068,7 +1133,10 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
           if (r < BT && grow < p.T) {
             const float *e = ebuf + rr * 33 + c4;
             const float4 base = accumulate ? old[g] : bias;
-            const float4 y = make_float4(base.x + e[0], base.y + e[1], base.z + e[2], base.w + e[3]);
+            const float sd = F8 ? p.s_delta : 1.f;
+            const float4 y = F8 ? make_float4(fmaf(e[0], sd, base.x), fmaf(e[1], sd, base.y), fmaf(e[2], sd, base.z),
+                                              fmaf(e[3], sd, base.w))
+                                : make_float4(base.x + e[0], base.y + e[1], base.z + e[2], base.w + e[3]);
             *reinterpret_cast<float4 *>(p.y_cache + grow * p.D + n) = y;
             if (p.out != nullptr)
               *reinterpret_cast<uint2 *>(p.out + grow * p.D + n) = make_uint2(cvt_bf16x2(y.x, y.y), cvt_bf16x2(y.z, y.w));
@@ -1149,7 +1217,47 @@ cudaError_t launch_down_bn(const MlpDownParams &p, const CUtensorMap &a, const C
   }
 }
 
+// out = bf16(y_cache) when a sparse step selects nothing
+cudaError_t y_to_out(const MlpDownParams &p, cudaStream_t s) {
+  if (p.out == nullptr) return cudaSuccess;
+  const int64_t n4 = static_cast<int64_t>(p.T) * p.D / 4;
+  y_to_out_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 16)), 256, 0, s>>>(
+      reinterpret_cast<const float4 *>(p.y_cache), reinterpret_cast<uint2 *>(p.out), n4);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_mlp_up_fp8(const MlpUpParams &p, const CUtensorMap &tm_x, cudaStream_t s) {
+  if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
+  if (p.Bt != 128 || p.mode != kUpDelta) return cudaErrorInvalidValue;
+  using C = UpCfg<128>;
+  cudaError_t e = set_smem(mlp_up_kernel<128, false, true>, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.nchunks, static_cast<int64_t>(sms) * C::kCtasPerSm);
+  // the W1^T tile map serves the refresh only; a sparse step gathers the rows itself
+  mlp_up_kernel<128, false, true><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, s>>>(tm_x, tm_x, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mlp_down_fp8(const MlpDownParams &p, const CUtensorMap &tm_a, cudaStream_t s) {
+  if (p.nb <= 0) return cudaSuccess;
+  if (p.k <= 0) return y_to_out(p, s);
+  if (p.Bt != 128 || p.bn != 256 || p.mode != kDownAccumulate) return cudaErrorInvalidValue;
+  using C = DownCfg<256>;
+  cudaError_t e = set_smem(mlp_down_kernel<128, 256, false, true>, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = std::min<int64_t>(static_cast<int64_t>(p.nb) * p.n_slices, static_cast<int64_t>(sms) * C::kCtasPerSm);
+  // the W2 tile map serves the refresh only; a sparse step gathers the rows itself
+  mlp_down_kernel<128, 256, false, true><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, s>>>(tm_a, tm_a, p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s) {
   if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
@@ -1163,13 +1271,7 @@ cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, con
                             cudaStream_t s) {
   if (p.nb <= 0) return cudaSuccess;
   const int kext = dense ? p.krows : p.k;
-  if (kext <= 0) {
-    if (p.out == nullptr) return cudaSuccess;
-    const int64_t n4 = static_cast<int64_t>(p.T) * p.D / 4;
-    y_to_out_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 16)), 256, 0, s>>>(
-        reinterpret_cast<const float4 *>(p.y_cache), reinterpret_cast<uint2 *>(p.out), n4);
-    return cudaGetLastError();
-  }
+  if (kext <= 0) return y_to_out(p, s);
   if (p.Bt == 128) return dense ? launch_down_bn<128, true>(p, tm_a, tm_w2, s) : launch_down_bn<128, false>(p, tm_a, tm_w2, s);
   if (p.Bt == 64) return dense ? launch_down_bn<64, true>(p, tm_a, tm_w2, s) : launch_down_bn<64, false>(p, tm_a, tm_w2, s);
   return cudaErrorInvalidValue;

@@ -174,6 +174,7 @@ typedef struct chipmunk_refresh_args {
 #define CHIPMUNK_OP_MLP_DELTA    1
 #define CHIPMUNK_OP_ATTN_DELTA   2
 #define CHIPMUNK_OP_REFRESH      3
+#define CHIPMUNK_OP_MLP_DELTA_FP8 4
 
 /*
  * Top-k column selection (post: Chipmunk "dynamically chooses which ones to
@@ -248,6 +249,63 @@ CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_down(const chipmunk_mlp_args *a,
  */
 #define CHIPMUNK_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_noalloc(const chipmunk_mlp_args *a, chipmunk_stream stream);
+
+/*
+ * FP8 form of the sparse MLP step (the post reports the method on an FP8
+ * FLUX.1-dev, sparsified, 1.1x over the fastest open-source implementation;
+ * the scaling scheme below is this library's). The gathered GEMMs run on e4m3
+ * operands (tcgen05 kind::f8f6f4, fp32 accumulation):
+ *   x[t][:]  ~ sx[t] * x8[t][:]          (per-token scale)
+ *   W1^T[c][:] ~ s1[c] * w1t8[c][:]      (per-hidden-unit scale)
+ *   W2[c][:] ~ s2[c] * w2_8[c][:]        (per-hidden-unit scale)
+ * For each block b and selected column c:
+ *   a = gelu(s1[c] sx[t] (x8[t] . w1t8[c]) + b1[c]);  delta = bf16(a) - a_cache[b][c];
+ *   code = e4m3(delta * g2[c])  with g2[c] = s2[c] / s_delta (rounded to nearest
+ *          even, saturated at +-448);
+ *   y_cache[t] += s_delta * sum_c code * w2_8[c];  a_cache[b][c] = bf16(a);
+ * then out = bf16(y_cache) if out is not NULL. s_delta is a static scale of
+ * the deltas chosen by the caller (deltas beyond 448 s_delta / s2[c]
+ * saturate). Use chipmunk_quantize_e4m3_rows for the codes and scales.
+ *   T, H    as for chipmunk_mlp_args; Bt must be 128; D a multiple of 256
+ *   x8      [T][D] e4m3 codes (bytes);  sx [T] fp32
+ *   w1t8    [H][D] e4m3;  s1 [H] fp32;  b1 [H] bf16
+ *   w2_8    [H][D] e4m3;  g2 [H] fp32;  s_delta > 0
+ *   idx, a_cache, y_cache, out: as for chipmunk_mlp_args
+ * Workspace: chipmunk_workspace_bytes(CHIPMUNK_OP_MLP_DELTA_FP8, a) bytes
+ * (nb * round_up(k,128) * 128 delta codes).
+ */
+typedef struct chipmunk_mlp_fp8_args {
+  int64_t T, D, H;
+  int32_t Bt, k;
+  const void *x8;
+  const float *sx;
+  const void *w1t8;
+  const float *s1;
+  const void *b1;
+  const void *w2_8;
+  const float *g2;
+  float s_delta;
+  int32_t *idx;
+  void *a_cache;
+  float *y_cache;
+  void *out;
+} chipmunk_mlp_fp8_args;
+
+CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_fp8(const chipmunk_mlp_fp8_args *a, void *ws, size_t ws_bytes,
+                                                    chipmunk_stream stream);
+
+/*
+ * Rows of bf16 values to e4m3 codes with one scale per row (the operands of
+ * chipmunk_mlp_delta_fp8: activations per token, weights per hidden unit).
+ * For each row r: amax = max |x[r][:]|, inv = 448 / amax and scale = amax / 448
+ * (fp32 divisions rounded to nearest; both 1 for an all-zero row), codes[r][i]
+ * = e4m3(x[r][i] * inv) (fp32 product, rounded to nearest even, saturated at
+ * +-448), scales[r] = scale, so that x ~ scale * code. Values must be finite.
+ *   x [rows][cols] bf16, codes [rows][cols] bytes, scales [rows] fp32;
+ *   cols a multiple of 16.
+ */
+CHIPMUNK_API chipmunk_status chipmunk_quantize_e4m3_rows(const void *x, int64_t rows, int64_t cols, void *codes,
+                                                         float *scales, chipmunk_stream stream);
 
 /*
  * Sparse attention step (post: attention output as a sum of scaled rows of V,

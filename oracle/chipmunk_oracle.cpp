@@ -96,6 +96,42 @@ uint16_t double_to_bf16(double x) {
   return static_cast<uint16_t>((static_cast<uint64_t>(u) + 0x7FFFu + lsb) >> 16);
 }
 
+// e4m3 (OCP FP8 E4M3: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+// infinities, S.1111.111 is NaN, the largest finite value 448 = 1.75 * 2^8,
+// subnormals m / 8 * 2^-6) from a float: rounded to nearest, ties to the even
+// code, magnitudes above 448 saturated to 448.
+uint8_t e4m3_encode(float x) {
+  if (std::isnan(x)) return 0x7F;
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(x));
+  if (a >= 448.0) return sign | 0x7E;
+  if (a < std::ldexp(1.0, -6)) {
+    // subnormal range: steps of 2^-9; 8 steps is the smallest normal, code 0x08
+    const double m = std::nearbyint(a * 512.0);
+    return sign | static_cast<uint8_t>(m);
+  }
+  int e2;
+  std::frexp(a, &e2);                  // a = f * 2^e2, f in [0.5, 1)
+  int e = e2 - 1;                      // a in [2^e, 2^(e+1))
+  double r = std::nearbyint(std::ldexp(a, 3 - e));   // in [8, 16]
+  if (r == 16.0) {
+    r = 8.0;
+    ++e;
+  }
+  const int be = e + 7;
+  const int m = static_cast<int>(r) - 8;
+  if (be > 15 || (be == 15 && m == 7)) return sign | 0x7E;
+  return sign | static_cast<uint8_t>((be << 3) | m);
+}
+
+double e4m3_decode(uint8_t c) {
+  const double sign = (c & 0x80) ? -1.0 : 1.0;
+  const int be = (c >> 3) & 15, m = c & 7;
+  if (be == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+  if (be == 0) return sign * std::ldexp(m / 8.0, -6);
+  return sign * std::ldexp(1.0 + m / 8.0, be - 7);
+}
+
 // ------------------------------------------------------------------ MLP pieces
 
 // GELU, tanh form (Hendrycks and Gimpel): the post's MLP non-linearity.
@@ -428,6 +464,83 @@ void or_mlp_refresh(const double *x, const double *w1t, const double *b1, const 
   std::vector<float> s32(nb * H);
   for (int64_t i = 0; i < nb * H; ++i) s32[i] = static_cast<float>(scores[i]);
   or_topk_cols(s32.data(), nb, H, k, idx);
+}
+
+// ------------------------------------------------------------------ FP8 form of the MLP step
+
+void or_e4m3_encode(const float *x, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(x[i]);
+}
+
+void or_e4m3_decode(const uint8_t *c, int64_t n, double *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_decode(c[i]);
+}
+
+// Rows of fp32 values (bf16 ones in practice) to e4m3 codes with one scale
+// per row: amax = max |x|, inv = 448 / amax and scale = amax / 448 (float
+// divisions; both 1 when amax is 0), code = e4m3(x * inv) (a float product),
+// so that x ~ scale * code.
+void or_quantize_rows_e4m3(const float *x, int64_t rows, int64_t cols, uint8_t *codes, float *scales) {
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.f;
+    for (int64_t i = 0; i < cols; ++i) amax = std::max(amax, std::fabs(x[r * cols + i]));
+    const float inv = amax > 0.f ? 448.f / amax : 1.f;
+    scales[r] = amax > 0.f ? amax / 448.f : 1.f;
+    for (int64_t i = 0; i < cols; ++i) {
+      const float prod = x[r * cols + i] * inv;
+      codes[r * cols + i] = e4m3_encode(prod);
+    }
+  }
+}
+
+// The FP8 form of one sparse MLP step (the library's own scaling scheme for
+// the post's FP8 FLUX result). Operands are e4m3 codes with scales: x[t] ~
+// sx[t] x8[t], W1^T[c] ~ s1[c] w1t8[c], W2[c] ~ s2[c] w2_8[c]. For each block
+// and selected column c: a = gelu(s1[c] sx[t] (x8[t] . w1t8[c]) + b1[c]); the
+// delta against the cache is taken from a rounded to bf16 (as it is stored),
+// multiplied by g2[c] = s2[c] / s_delta as floats and rounded to an e4m3 code;
+// the cached output gains s_delta * sum_c code * w2_8[c]. A_new takes a.
+void or_mlp_delta_fp8(const uint8_t *x8, const float *sx, const uint8_t *w1t8, const float *s1, const double *b1,
+                      const uint8_t *w2_8, const float *g2, float s_delta, const int32_t *idx, int64_t k,
+                      const double *A_cache, const double *Y_cache, int64_t T, int64_t D, int64_t H, int64_t Bt,
+                      double *A_new, double *Y_new) {
+  std::memcpy(A_new, A_cache, sizeof(double) * T * H);
+  std::memcpy(Y_new, Y_cache, sizeof(double) * T * D);
+  if (k == 0) return;
+  std::vector<double> xd(T * D), w1d(H * D), w2d(H * D);
+  for (int64_t i = 0; i < T * D; ++i) xd[i] = e4m3_decode(x8[i]);
+  for (int64_t i = 0; i < H * D; ++i) w1d[i] = e4m3_decode(w1t8[i]);
+  for (int64_t i = 0; i < H * D; ++i) w2d[i] = e4m3_decode(w2_8[i]);
+  parallel_for(block_count(T, Bt), [&](int64_t b) {
+    int64_t blk0, blk1;
+    block_range(b, T, Bt, &blk0, &blk1);
+    const int32_t *S = idx + b * k;
+    std::vector<const double *> w2rows(k);
+    for (int64_t j = 0; j < k; ++j) w2rows[j] = w2d.data() + static_cast<int64_t>(S[j]) * D;
+    std::vector<double> xt(D * kRows), u(kRows), code(kRows * k), change(kRows * D);
+    const std::vector<double> no_bias(H, 0.0);
+    for (int64_t r0 = blk0; r0 < blk1; r0 += kRows) {
+      const int64_t r1 = std::min(r0 + kRows, blk1), nr = r1 - r0;
+      transpose_rows(xd.data(), r0, r1, D, xt.data());
+      for (int64_t j = 0; j < k; ++j) {
+        const int64_t c = S[j];
+        preactivation(xt.data(), nr, w1d.data(), no_bias.data(), D, c, u.data());   // x8[t] . w1t8[c]
+        for (int64_t r = 0; r < nr; ++r) {
+          const double an = gelu(u[r] * s1[c] * sx[r0 + r] + b1[c]);
+          const double stored = bf16_to_double(double_to_bf16(an));
+          const float d = static_cast<float>(stored - A_cache[(r0 + r) * H + c]);
+          code[r * k + j] = e4m3_decode(e4m3_encode(d * g2[c]));
+          A_new[(r0 + r) * H + c] = an;
+        }
+      }
+      std::fill(change.begin(), change.end(), 0.0);
+      weighted_row_sums(code.data(), k, nr, w2rows.data(), k, D, change.data(), D);
+      for (int64_t r = 0; r < nr; ++r) {
+        double *yr = Y_new + (r0 + r) * D;
+        for (int64_t n = 0; n < D; ++n) yr[n] += static_cast<double>(s_delta) * change[r * D + n];
+      }
+    }
+  });
 }
 
 // ------------------------------------------------------------------ attention

@@ -146,6 +146,88 @@ def mlp_refresh(x, W1, b1, W2, b2, A_old, Bt, k, first_step):
     return dict(a=a, y=y, scores=scores, idx=topk_cols(f32(scores), k))
 
 
+# --------------------------------------------------------------------------- FP8 form of the MLP step
+
+def e4m3_encode(x32: np.ndarray) -> np.ndarray:
+    """fp32 values -> e4m3 codes (OCP FP8 E4M3: bias 7, 3 mantissa bits, no infinities, NaN S.1111.111,
+    largest finite 448): nearest representable value, ties to the even code, magnitudes above 448
+    saturated to 448."""
+    x = np.asarray(x32, dtype=np.float32).astype(np.float64)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    flat, res = x.reshape(-1), out.reshape(-1)
+    for i, v in enumerate(flat):
+        if math.isnan(v):
+            res[i] = 0x7F
+            continue
+        sign = 0x80 if math.copysign(1.0, v) < 0 else 0
+        a = abs(v)
+        if a >= 448.0:
+            res[i] = sign | 0x7E
+            continue
+        if a < 2.0 ** -6:
+            res[i] = sign | int(round(a * 512.0))      # round() is half-to-even
+            continue
+        e = math.floor(math.log2(a))
+        if 2.0 ** e > a:                              # guard the logarithm's rounding
+            e -= 1
+        elif 2.0 ** (e + 1) <= a:
+            e += 1
+        r = round(a / 2.0 ** (e - 3))
+        if r == 16:
+            r, e = 8, e + 1
+        be, m = e + 7, r - 8
+        res[i] = sign | (0x7E if be > 15 or (be == 15 and m == 7) else (be << 3) | m)
+    return out
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """e4m3 codes -> exact float64 values (NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    be, m = (c >> 3) & 15, c & 7
+    val = np.where(be == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(be - 7.0))
+    return np.where((be == 15) & (m == 7), np.nan, sign * val)
+
+
+def quantize_rows_e4m3(x):
+    """Rows of fp32 values to e4m3 codes with one scale per row, in float arithmetic:
+    amax = max |x|, inv = 448 / amax, scale = amax / 448 (both 1 when amax is 0),
+    code = e4m3(x * inv), so that x ~ scale * code. Returns (codes uint8, scales float32)."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float32))
+    amax = np.abs(x).max(axis=1)
+    pos = amax > 0
+    safe = np.where(pos, amax, np.float32(1.0)).astype(np.float32)
+    inv = np.where(pos, np.float32(448.0) / safe, np.float32(1.0)).astype(np.float32)
+    scales = np.where(pos, safe / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    return e4m3_encode((x * inv[:, None]).astype(np.float32)), scales
+
+
+def mlp_delta_fp8(x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt):
+    """One sparse MLP step on e4m3 operands (the library's own scaling scheme for the post's FP8
+    FLUX result): x[t] ~ sx[t] x8[t], W1^T[c] ~ s1[c] w1t8[c], W2[c] ~ s2[c] w2_8[c]. For each block
+    and selected column c: a = gelu(s1[c] sx[t] (x8[t] . w1t8[c]) + b1[c]); the delta against the
+    cache is taken from a rounded to bf16 (as stored), multiplied by g2[c] = s2[c] / s_delta as
+    floats and rounded to an e4m3 code; the cached output gains s_delta * sum_c code * w2_8[c].
+    Returns (A_new, Y_new); A_new takes a."""
+    xd, w1d, w2d = e4m3_decode(x8), e4m3_decode(w1t8), e4m3_decode(w2_8)
+    sx, s1, g2 = (np.asarray(a, dtype=np.float32) for a in (sx, s1, g2))
+    T = xd.shape[0]
+    A_new = np.array(A_cache, dtype=np.float64, copy=True)
+    Y_new = np.array(Y_cache, dtype=np.float64, copy=True)
+    for b, r0, r1 in blocks(T, Bt):
+        S = np.asarray(idx[b], dtype=np.int64)
+        if S.size == 0:
+            continue
+        u = (xd[r0:r1] @ w1d[S].T) * s1[S].astype(np.float64)[None, :] * sx[r0:r1].astype(np.float64)[:, None]
+        a = gelu_tanh(u + np.asarray(b1, dtype=np.float64)[S][None, :])
+        stored = bf16_decode(bf16_round(a))
+        d = (stored - A_cache[r0:r1][:, S]).astype(np.float32)
+        code = e4m3_decode(e4m3_encode((d * g2[S][None, :]).astype(np.float32)))
+        Y_new[r0:r1] += np.float64(np.float32(s_delta)) * (code @ w2d[S, :])
+        A_new[r0:r1, S] = a
+    return A_new, Y_new
+
+
 # --------------------------------------------------------------------------- selection
 
 def ordered_key(s32: np.ndarray) -> np.ndarray:

@@ -55,6 +55,7 @@ _D = ctypes.POINTER(ctypes.c_double)
 _I32 = ctypes.POINTER(ctypes.c_int32)
 _U16 = ctypes.POINTER(ctypes.c_uint16)
 _U32 = ctypes.POINTER(ctypes.c_uint32)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
 _F32 = ctypes.POINTER(ctypes.c_float)
 _I64 = ctypes.c_int64
 _SIGS = {
@@ -72,6 +73,11 @@ _SIGS = {
     "or_ordered_key": (None, [_F32, _I64, _U32]),
     "or_topk_cols": (None, [_F32, _I64, _I64, _I64, _I32]),
     "or_mlp_refresh": (None, [_D, _D, _D, _D, _D, _D, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _D, _D, _D, _I32]),
+    "or_e4m3_encode": (None, [_F32, _I64, _U8]),
+    "or_e4m3_decode": (None, [_U8, _I64, _D]),
+    "or_quantize_rows_e4m3": (None, [_F32, _I64, _I64, _U8, _F32]),
+    "or_mlp_delta_fp8": (None, [_U8, _F32, _U8, _F32, _D, _U8, _F32, ctypes.c_float, _I32, _I64, _D, _D, _I64, _I64,
+                                _I64, _I64, _D, _D]),
     "or_attn_partial": (None, [_D, _I64, _D, _D, _I64, _I64, ctypes.c_double, _D, _D, _D]),
     "or_merge_partials": (None, [_D, _D, _D, _D, _D, _D, _I64, _I64, _D, _D, _D]),
     "or_finish": (None, [_D, _D, _I64, _I64, _D]),
@@ -202,6 +208,45 @@ class CppOracle:
                                 _p(idx, _I32))
         return dict(a=a, y=y, scores=scores, idx=idx)
 
+    # ---------------------------------------------------------------- FP8
+
+    def e4m3_encode(self, x32):
+        x = np.ascontiguousarray(x32, dtype=np.float32)
+        out = np.empty(x.shape, dtype=np.uint8)
+        self.lib.or_e4m3_encode(_p(x, _F32), x.size, _p(out, _U8))
+        return out
+
+    def e4m3_decode(self, codes):
+        c = np.ascontiguousarray(codes, dtype=np.uint8)
+        out = np.empty(c.shape)
+        self.lib.or_e4m3_decode(_p(c, _U8), c.size, _p(out, _D))
+        return out
+
+    def quantize_rows_e4m3(self, x):
+        x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float32)
+        rows, cols = x.shape
+        codes = np.empty((rows, cols), dtype=np.uint8)
+        scales = np.empty(rows, dtype=np.float32)
+        self.lib.or_quantize_rows_e4m3(_p(x, _F32), rows, cols, _p(codes, _U8), _p(scales, _F32))
+        return codes, scales
+
+    def mlp_delta_fp8(self, x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt):
+        x8 = np.ascontiguousarray(x8, dtype=np.uint8)
+        w1t8 = np.ascontiguousarray(w1t8, dtype=np.uint8)
+        w2_8 = np.ascontiguousarray(w2_8, dtype=np.uint8)
+        sx, s1, g2 = (np.ascontiguousarray(a, dtype=np.float32) for a in (sx, s1, g2))
+        b1 = _f64(b1)
+        A, Y = _f64(A_cache), _f64(Y_cache)
+        T, D = x8.shape
+        H = w1t8.shape[0]
+        nb = len(self.blocks(T, Bt))
+        ix = np.ascontiguousarray(np.asarray(idx, dtype=np.int32).reshape(nb, -1))
+        A_new, Y_new = np.empty_like(A), np.empty_like(Y)
+        self.lib.or_mlp_delta_fp8(_p(x8, _U8), _p(sx, _F32), _p(w1t8, _U8), _p(s1, _F32), _p(b1, _D), _p(w2_8, _U8),
+                                  _p(g2, _F32), float(s_delta), _p(ix, _I32), ix.shape[1], _p(A, _D), _p(Y, _D), T, D,
+                                  H, int(Bt), _p(A_new, _D), _p(Y_new, _D))
+        return A_new, Y_new
+
     # ---------------------------------------------------------------- selection
 
     def ordered_key(self, s32):
@@ -323,6 +368,7 @@ class CppOracle:
 
 
 FUNCTIONS = ("bf16_decode", "bf16_round", "f32", "k_from_density", "blocks", "gelu_tanh", "dense_mlp", "mlp_delta",
+             "e4m3_encode", "e4m3_decode", "quantize_rows_e4m3", "mlp_delta_fp8",
              "mlp_scores", "mlp_refresh", "ordered_key", "topk_cols", "attn_partial", "merge_partials", "finish",
              "attn_delta", "compact_partial", "attn_delta_compact", "dense_attention", "attn_mass_rows", "attn_mass",
              "complement_partial", "attn_refresh")

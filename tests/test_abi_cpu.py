@@ -45,7 +45,7 @@ def test_struct_layouts_match_the_header(cm, tmp_path):
     if gcc is None:
         pytest.skip("no C compiler")
     structs = {"chipmunk_mlp_args": cm.MlpArgs, "chipmunk_attn_args": cm.AttnArgs,
-               "chipmunk_refresh_args": cm.RefreshArgs}
+               "chipmunk_refresh_args": cm.RefreshArgs, "chipmunk_mlp_fp8_args": cm.MlpFp8Args}
     lines = ["#include <stddef.h>", "#include <stdio.h>", "#include \"chipmunk.h\"", "int main(void) {"]
     for cname, py in structs.items():
         lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
@@ -149,3 +149,37 @@ def test_status_constants_match_the_header(cm):
         assert m and int(m.group(1)) == getattr(cm, name), name
     m = re.search(r"#define CHIPMUNK_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
     assert m and (int(m.group(1)) << int(m.group(2))) == cm.NOALLOC_SCRATCH_BYTES
+
+
+def _fp8_args(cm, **kw):
+    base = dict(T=300, D=256, H=700, Bt=128, k=128, x8=0x1000, sx=0x2000, w1t8=0x3000, s1=0x4000, b1=0x5000,
+                w2_8=0x6000, g2=0x7000, s_delta=1e-4, idx=0x8000, a_cache=0x9000, y_cache=0xa000, out=0)
+    base.update(kw)
+    return cm.MlpFp8Args(**base)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("D", 128, "ERR_SHAPE"), ("D", 384, "ERR_SHAPE"), ("Bt", 64, "ERR_SHAPE"), ("k", 701, "ERR_INVALID_ARG"),
+    ("s_delta", 0.0, "ERR_INVALID_ARG"), ("s_delta", -1.0, "ERR_INVALID_ARG"), ("sx", 0, "ERR_INVALID_ARG"),
+    ("g2", 0x7004, "ERR_ALIGNMENT"),
+])
+def test_mlp_delta_fp8_rejects_bad_arguments_on_the_host(cm, field, value, status):
+    lib = cm.load_library()
+    a = _fp8_args(cm, **{field: value})
+    assert lib.chipmunk_mlp_delta_fp8(ctypes.byref(a), None, 0, None) == getattr(cm, status), lib.chipmunk_last_error()
+
+
+def test_mlp_delta_fp8_workspace(cm):
+    lib = cm.load_library()
+    a = _fp8_args(cm)
+    assert lib.chipmunk_workspace_bytes(cm.OP_MLP_DELTA_FP8, ctypes.byref(a)) == 3 * 128 * 128   # one byte per delta
+    assert lib.chipmunk_mlp_delta_fp8(ctypes.byref(a), None, 0, None) == cm.ERR_WORKSPACE
+
+
+def test_quantize_rejects_bad_arguments_on_the_host(cm):
+    lib = cm.load_library()
+    q = lib.chipmunk_quantize_e4m3_rows
+    assert q(ctypes.c_void_p(0x1000), 4, 24, ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000), None) == cm.ERR_SHAPE
+    assert q(ctypes.c_void_p(0x1008), 4, 32, ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000), None) == cm.ERR_ALIGNMENT
+    assert q(None, 4, 32, ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000), None) == cm.ERR_INVALID_ARG
+    assert q(None, 0, 32, None, None, None) == cm.OK

@@ -145,3 +145,30 @@ def test_thread_count_does_not_change_results():
     assert C.threads() == before
     assert np.array_equal(outs[0][0][0], outs[1][0][0]) and np.array_equal(outs[0][0][1], outs[1][0][1])
     assert np.array_equal(outs[0][1], outs[1][1])
+
+
+def test_fp8_functions():
+    codes = np.arange(256, dtype=np.uint32).astype(np.uint8)
+    a, b = C.e4m3_decode(codes), N.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(a), np.isnan(b)) and np.array_equal(a[~np.isnan(a)], b[~np.isnan(b)])
+    x = (g.standard_normal(30000) * 10.0 ** g.integers(-5, 4, 30000)).astype(np.float32)
+    x[:6] = [0.0, -0.0, 448.0, 1e9, -np.inf, 2.0 ** -10]
+    assert np.array_equal(C.e4m3_encode(x), N.e4m3_encode(x))
+    rows = x.reshape(30, 1000).copy()
+    rows[0, 4] = -1e9                                    # quantised rows hold finite values
+    rows[3] = 0.0
+    qc, qn = C.quantize_rows_e4m3(rows), N.quantize_rows_e4m3(rows)
+    assert np.array_equal(qc[0], qn[0]) and np.array_equal(qc[1], qn[1])
+    T, D, H, Bt, k = 40, 48, 70, 16, 30
+    x8, sx = N.quantize_rows_e4m3(g.standard_normal((T, D)).astype(np.float32))
+    w1t8, s1 = N.quantize_rows_e4m3((g.standard_normal((H, D)) / 7).astype(np.float32))
+    w2_8, s2 = N.quantize_rows_e4m3((g.standard_normal((H, D)) / 8).astype(np.float32))
+    b1 = 0.02 * g.standard_normal(H)
+    A = N.bf16_decode(N.bf16_round(0.5 * g.standard_normal((T, H))))
+    Y = g.standard_normal((T, D))
+    idx = np.sort(np.stack([g.choice(H, k, replace=False) for _ in range(3)]), axis=1).astype(np.int32)
+    g2 = (s2 / np.float32(1e-4)).astype(np.float32)
+    rc = C.mlp_delta_fp8(x8, sx, w1t8, s1, b1, w2_8, g2, np.float32(1e-4), idx, A, Y, Bt)
+    rn = N.mlp_delta_fp8(x8, sx, w1t8, s1, b1, w2_8, g2, np.float32(1e-4), idx, A, Y, Bt)
+    for got, ref, what in zip(rc, rn, ("A", "Y")):
+        close(got, ref, f"mlp_delta_fp8 {what}")

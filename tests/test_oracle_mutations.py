@@ -251,7 +251,48 @@ def _bf16_decode_low_half(bits):
         return (np.asarray(bits, dtype=np.uint32) << np.uint32(15)).view(np.float32).astype(np.float64)
 
 
+def _e4m3_truncate(x32):
+    x = np.asarray(x32, dtype=np.float32)
+    out = ORIG_E4M3(x)
+    back = OC.e4m3_decode(out)
+    over = np.abs(back) > np.abs(x.astype(np.float64))      # rounded away from zero: step back one code
+    return np.where(over & (out & 0x7F > 0), out - 1, out).astype(np.uint8)
+
+
+def _e4m3_no_saturation(x32):
+    x = np.asarray(x32, dtype=np.float32)
+    out = ORIG_E4M3(x)
+    return np.where(np.abs(x) > 448.0, np.uint8(0x7F), out).astype(np.uint8)
+
+
+def _quantize_scale_off_by_one_code(x):
+    codes, scales = ORIG_QUANT(x)
+    return codes, (scales * np.float32(1.0625)).astype(np.float32)
+
+
+def _fp8_no_delta_scale(x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt):
+    return ORIG_FP8(x8, sx, w1t8, s1, b1, w2_8, g2, np.float32(1.0), idx, A_cache, Y_cache, Bt)
+
+
+def _fp8_no_g2(x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt):
+    return ORIG_FP8(x8, sx, w1t8, s1, b1, w2_8, np.ones_like(np.asarray(g2)), s_delta, idx, A_cache, Y_cache, Bt)
+
+
+def _fp8_no_s1(x8, sx, w1t8, s1, b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt):
+    return ORIG_FP8(x8, sx, w1t8, np.ones_like(np.asarray(s1)), b1, w2_8, g2, s_delta, idx, A_cache, Y_cache, Bt)
+
+
+ORIG_E4M3 = OC.e4m3_encode
+ORIG_QUANT = OC.quantize_rows_e4m3
+ORIG_FP8 = OC.mlp_delta_fp8
+
 MUTATIONS = {
+    "e4m3_encode: truncation instead of nearest-even": ("e4m3_encode", _e4m3_truncate),
+    "e4m3_encode: no saturation at 448": ("e4m3_encode", _e4m3_no_saturation),
+    "quantize_rows_e4m3: scale off": ("quantize_rows_e4m3", _quantize_scale_off_by_one_code),
+    "mlp_delta_fp8: delta scale dropped": ("mlp_delta_fp8", _fp8_no_delta_scale),
+    "mlp_delta_fp8: g2 not applied": ("mlp_delta_fp8", _fp8_no_g2),
+    "mlp_delta_fp8: W1 row scale dropped": ("mlp_delta_fp8", _fp8_no_s1),
     "gelu_tanh: cubic term dropped": ("gelu_tanh", _gelu_no_cubic),
     "gelu_tanh: sign of tanh flipped": ("gelu_tanh", _gelu_sign),
     "mlp_delta: delta sign flipped": ("mlp_delta", _mlp_delta_sign),
@@ -302,7 +343,8 @@ CPP_MUTATIONS = {
     "preactivation: bias b1 dropped": ("u[r] = acc[r] + b1[c];", "u[r] = acc[r];"),
     "preactivation: first input feature skipped": ("  for (int64_t d = 0; d < D; ++d) {\n    const double *xd",
                                                    "  for (int64_t d = 1; d < D; ++d) {\n    const double *xd"),
-    "mlp_delta: cache not written back": ("A_new[(r0 + r) * H + c] = an;", "(void)an;"),
+    "mlp_delta: cache not written back": ("delta[r * k + j] = an - A_cache[(r0 + r) * H + c];\n          A_new[(r0 + r) * H + c] = an;",
+                                          "delta[r * k + j] = an - A_cache[(r0 + r) * H + c];"),
     "weighted_row_sums: last term of every chunk dropped": ("const int64_t j1 = std::min(j0 + kTerms, ncoef);",
                                                             "const int64_t j1 = std::min(j0 + kTerms - 1, ncoef);"),
     "weighted_row_sums: ragged output tail skipped": ("for (int64_t e = 0; e < nn; ++e) o[e] += coef[r * ldc + j] * rows[j][n0 + e];",
@@ -339,6 +381,14 @@ CPP_MUTATIONS = {
     "blocks: short last block dropped": ("int64_t block_count(int64_t T, int64_t Bt) { return (T + Bt - 1) / Bt; }",
                                          "int64_t block_count(int64_t T, int64_t Bt) { return T / Bt; }"),
     "bf16_decode: bits shifted by 15": ("static_cast<uint32_t>(bits) << 16;", "static_cast<uint32_t>(bits) << 15;"),
+    "e4m3: subnormals truncated": ("const double m = std::nearbyint(a * 512.0);", "const double m = std::floor(a * 512.0);"),
+    "e4m3: normals truncated": ("double r = std::nearbyint(std::ldexp(a, 3 - e));", "double r = std::floor(std::ldexp(a, 3 - e));"),
+    "e4m3: exponent bias 8": ("return sign | static_cast<uint8_t>((be << 3) | m);", "return sign | static_cast<uint8_t>(((be + 1) << 3) | m);"),
+    "e4m3 decode: subnormal scale 2^-7": ("if (be == 0) return sign * std::ldexp(m / 8.0, -6);", "if (be == 0) return sign * std::ldexp(m / 8.0, -7);"),
+    "quantize_rows: inverse scale 1/448": ("const float inv = amax > 0.f ? 448.f / amax : 1.f;", "const float inv = amax > 0.f ? 1.f / amax : 1.f;"),
+    "mlp_delta_fp8: delta from the unrounded activation": ("const double stored = bf16_to_double(double_to_bf16(an));", "const double stored = an;"),
+    "mlp_delta_fp8: delta scale dropped": ("yr[n] += static_cast<double>(s_delta) * change[r * D + n];", "yr[n] += change[r * D + n];"),
+    "mlp_delta_fp8: token scale dropped": ("const double an = gelu(u[r] * s1[c] * sx[r0 + r] + b1[c]);", "const double an = gelu(u[r] * s1[c] + b1[c]);"),
 }
 
 

@@ -151,6 +151,127 @@ def test_k_fixture_from_pages_sparsity():
         assert O.k_from_density(int(n), int(permille)) == int(k), name
 
 
+# --------------------------------------------------------------------------- FP8
+
+def test_e4m3_codes_fixture_and_roundtrip():
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "e4m3_codes.txt")) if ln.strip() and not ln.startswith("#")]
+    for code, expr in rows:
+        val = float(eval(expr))  # fixture holds plain arithmetic only
+        got = O.e4m3_decode(np.array([int(code, 16)], dtype=np.uint8))[0]
+        assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val), (code, got, val)
+        assert int(O.e4m3_encode(np.array([val], dtype=np.float32))[0]) == int(code, 16), code
+    codes = np.arange(256, dtype=np.uint32).astype(np.uint8)
+    vals = O.e4m3_decode(codes)
+    nan = np.isnan(vals)
+    assert sorted(codes[nan].tolist()) == [0x7F, 0xFF]
+    np.testing.assert_array_equal(O.e4m3_encode(vals[~nan].astype(np.float32)), codes[~nan])
+
+
+def test_e4m3_rounds_to_nearest_even_and_saturates():
+    pos = np.arange(0, 0x7F, dtype=np.uint32).astype(np.uint8)   # 0 .. 448, increasing
+    v = O.e4m3_decode(pos)
+    assert np.all(np.diff(v) > 0)
+    for lo in range(len(v) - 1):
+        a, b = v[lo], v[lo + 1]
+        mid = np.float32((a + b) / 2)                    # at most 5 significant bits: exact
+        assert float(mid) == (a + b) / 2
+        want = lo if lo % 2 == 0 else lo + 1              # the even code (lowest mantissa bit 0)
+        assert int(O.e4m3_encode(np.array([mid]))[0]) == want, (a, b)
+        assert int(O.e4m3_encode(np.array([np.nextafter(mid, np.float32(0))]))[0]) == lo
+        assert int(O.e4m3_encode(np.array([np.nextafter(mid, np.float32(1e9))]))[0]) == lo + 1
+        assert int(O.e4m3_encode(np.array([-mid]))[0]) == want | 0x80
+    big = np.array([448.0, 449.0, 464.0, 1e6, np.inf], dtype=np.float32)
+    assert O.e4m3_encode(big).tolist() == [0x7E] * 5
+    assert O.e4m3_encode(-big).tolist() == [0xFE] * 5
+
+
+def test_quantize_rows_e4m3():
+    g = np.random.default_rng(21)
+    x = (g.standard_normal((6, 96)) * 10.0 ** g.integers(-3, 3, (6, 1))).astype(np.float32)
+    x[4] = 0.0
+    x[5, :] = 1e-3
+    x[5, 7] = -7.5                                       # one large value sets the row's scale
+    codes, scales = O.quantize_rows_e4m3(x)
+    assert codes.shape == x.shape and codes.dtype == np.uint8 and scales.dtype == np.float32
+    for r in range(6):
+        amax = np.float32(np.abs(x[r]).max())
+        if amax == 0:
+            assert scales[r] == 1.0 and not codes[r].any()
+            continue
+        assert scales[r] == amax / np.float32(448.0)
+        j = int(np.abs(x[r]).argmax())
+        assert codes[r, j] in (0x7E, 0xFE)               # the largest magnitude lands on +-448
+        back = O.e4m3_decode(codes[r]) * float(scales[r])
+        # within half an e4m3 step (2^-4 relative) of the value, or of the subnormal step for tiny ones
+        bound = 2.0 ** -4 * np.abs(x[r]) + 2.0 ** -10 * float(scales[r]) + 1e-6 * float(amax)
+        assert np.all(np.abs(back - x[r]) <= bound), r
+
+
+def _fp8_case(T=20, D=32, H=50, k=12, Bt=8, seed=3):
+    g = np.random.default_rng(seed)
+    x8, sx = O.quantize_rows_e4m3(g.standard_normal((T, D)).astype(np.float32))
+    w1t8, s1 = O.quantize_rows_e4m3((g.standard_normal((H, D)) / math.sqrt(D)).astype(np.float32))
+    w2_8, s2 = O.quantize_rows_e4m3((g.standard_normal((H, D)) / math.sqrt(H)).astype(np.float32))
+    b1 = 0.02 * g.standard_normal(H)
+    A = O.bf16_decode(O.bf16_round(0.5 * g.standard_normal((T, H))))
+    Y = g.standard_normal((T, D))
+    nb = (T + Bt - 1) // Bt
+    idx = np.sort(np.stack([g.choice(H, k, replace=False) for _ in range(nb)]), axis=1).astype(np.int32)
+    s_delta = np.float32(1e-4)
+    g2 = (s2 / s_delta).astype(np.float32)
+    return dict(x8=x8, sx=sx, w1t8=w1t8, s1=s1, b1=b1, w2_8=w2_8, s2=s2, g2=g2, s_delta=s_delta, A=A, Y=Y, idx=idx,
+                Bt=Bt, T=T, D=D, H=H)
+
+
+def test_mlp_delta_fp8_written_out():
+    c = _fp8_case()
+    A1, Y1 = O.mlp_delta_fp8(c["x8"], c["sx"], c["w1t8"], c["s1"], c["b1"], c["w2_8"], c["g2"], c["s_delta"], c["idx"],
+                             c["A"], c["Y"], c["Bt"])
+    xd, w1d, w2d = O.e4m3_decode(c["x8"]), O.e4m3_decode(c["w1t8"]), O.e4m3_decode(c["w2_8"])
+    for b, r0, r1 in [(0, 0, 8), (1, 8, 16), (2, 16, 20)]:
+        for t in range(r0, r1):
+            change = [0.0] * c["D"]
+            for col in c["idx"][b]:
+                dot = 0.0
+                for d in range(c["D"]):
+                    dot += xd[t, d] * w1d[col, d]
+                u = dot * float(c["s1"][col]) * float(c["sx"][t]) + c["b1"][col]
+                a = 0.5 * u * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+                assert abs(A1[t, col] - a) <= 1e-12 * max(1.0, abs(a))
+                stored = O.bf16_decode(O.bf16_round(np.array([a])))[0]
+                dlt = np.float32(stored - c["A"][t, col]) * np.float32(c["g2"][col])
+                q = O.e4m3_decode(O.e4m3_encode(np.array([dlt], dtype=np.float32)))[0]
+                for n in range(c["D"]):
+                    change[n] += q * w2d[col, n]
+            for n in range(c["D"]):
+                assert abs(Y1[t, n] - (c["Y"][t, n] + float(c["s_delta"]) * change[n])) <= 1e-12 * max(1.0, abs(Y1[t, n]))
+    sel = np.zeros((c["T"], c["H"]), dtype=bool)
+    for b, r0, r1 in [(0, 0, 8), (1, 8, 16), (2, 16, 20)]:
+        sel[r0:r1, c["idx"][b]] = True
+    np.testing.assert_array_equal(A1[~sel], c["A"][~sel])
+
+
+def test_mlp_delta_fp8_no_columns_and_the_unquantised_step():
+    c = _fp8_case()
+    none = np.zeros((3, 0), dtype=np.int32)
+    A0, Y0 = O.mlp_delta_fp8(c["x8"], c["sx"], c["w1t8"], c["s1"], c["b1"], c["w2_8"], c["g2"], c["s_delta"], none,
+                             c["A"], c["Y"], c["Bt"])
+    np.testing.assert_array_equal(A0, c["A"])
+    np.testing.assert_array_equal(Y0, c["Y"])
+    # against the bf16-path step on the dequantised operands: the same activations, and outputs within
+    # the rounding of the deltas to e4m3 (half a step, 2^-4 relative, per term)
+    A1, Y1 = O.mlp_delta_fp8(c["x8"], c["sx"], c["w1t8"], c["s1"], c["b1"], c["w2_8"], c["g2"], c["s_delta"], c["idx"],
+                             c["A"], c["Y"], c["Bt"])
+    x = O.e4m3_decode(c["x8"]) * c["sx"].astype(np.float64)[:, None]
+    W1 = (O.e4m3_decode(c["w1t8"]) * c["s1"].astype(np.float64)[:, None]).T
+    W2 = O.e4m3_decode(c["w2_8"]) * c["s2"].astype(np.float64)[:, None]
+    A2, Y2 = O.mlp_delta(x, W1, c["b1"], W2, c["idx"], c["A"], c["Y"], c["Bt"])
+    np.testing.assert_allclose(A1, A2, rtol=1e-12, atol=1e-12)
+    dY = np.abs((Y1 - c["Y"]) - (Y2 - c["Y"]))
+    ref = np.abs(Y2 - c["Y"])
+    assert dY.max() <= 0.1 * ref.max() and dY.max() > 0
+
+
 # --------------------------------------------------------------------------- MLP
 
 def _mlp_case(T=24, D=8, H=20, seed=0):
