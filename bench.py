@@ -245,9 +245,10 @@ def cpu_baseline(w):
 # ---------------------------------------------------------------- GPU arm
 
 class Layer:
-    """Device-resident FLUX-shaped layer: weights, two drifted inputs, caches and selections."""
+    """Device-resident layer of the workload `w`: weights, two drifted inputs, caches and selections.
+    With keep_mass the attention refresh also keeps the mass [h][nb][T] (the standalone top-k rows use it)."""
 
-    def __init__(self, w, dev, seed):
+    def __init__(self, w, dev, seed, keep_mass=False):
         import torch
         from dynamic_column_sparse_b200 import chipmunk as cm
         self.w, self.dev, self.cm = w, dev, cm
@@ -281,9 +282,10 @@ class Layer:
         self.l_c = torch.empty((h, T), dtype=f32, device=dev)
         self.acc_c = torch.empty((h, T, d), dtype=f32, device=dev)
         self.o = torch.empty((T, h, d), dtype=torch.bfloat16, device=dev)
-        self.mass = torch.empty((h, self.nb, T), dtype=f32, device=dev)
+        self.mass = torch.empty((h, self.nb, T), dtype=f32, device=dev) if keep_mass else None
         self.ws = torch.empty(cm.mlp_workspace_bytes(T, H, self.kc, Bt), dtype=torch.uint8, device=dev)
-        self.attn_ws = torch.empty(h * T * 4, dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(cm.attn_refresh_workspace_bytes(T, h, self.kk, keep_mass), dtype=torch.uint8,
+                                   device=dev)
         self.x_prev, self.qkv_prev = x_prev, qkv_prev
         self.refresh()
 
@@ -595,7 +597,7 @@ def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
     if "workloads" in groups:
         hunyuan_refresh_rows(L, w, rows, gbs, flush, torch, cm)
     wf = dict(FLUX)
-    LF = Layer(wf, L.dev, seed=77)
+    LF = Layer(wf, L.dev, seed=77, keep_mass=True)
     T, D, H, h = wf["T"], wf["D"], wf["H"], wf["heads"]
     if "workloads" in groups:
         # the same sparse step at the pages' two FLUX.1-dev workloads: 1280x768 (80 x 48 latent
@@ -637,23 +639,30 @@ def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
 
 
 def hunyuan_refresh_rows(L, w, rows, gbs, flush, torch, cm):
-    """a5 at the HunyuanVideo layer: the dense MLP refresh, and the attention refresh (dense pass,
-    attention mass, top-k over h * nb rows of T, complement pass), with the top-k alone timed too."""
+    """a5 at the HunyuanVideo layer: the dense MLP refresh, and the attention refresh (dense pass, the
+    attention mass with its top-k in one kernel, complement pass). For comparison the attention refresh
+    is also timed keeping the mass in HBM, and the standalone top-k over that kept mass."""
     T, D, H, h, d = w["T"], w["D"], w["H"], w["heads"], w["d"]
     ms_mlp = time_events(lambda: cm.mlp_refresh(L.x_prev, L.w1t, L.b1, L.w2, L.b2, L.a_cache, L.y_cache, L.idx,
                                                 L.mlp_scores, L.out, Bt=w["Bt"]), 3, flush, torch)
     q, k, v = L.qkv_prev
-    ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, L.mass,
+    ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, None,
                                                   scale=1 / math.sqrt(d), workspace=L.attn_ws), 3, flush, torch)
-    mass2 = L.mass.view(h * L.nb, T)
-    aidx2 = L.aidx.view(h * L.nb, L.kk)
-    ms_topk = time_events(lambda: cm.topk_cols(mass2, L.kk, out=aidx2), 3, flush, torch)
+    mass = torch.empty((h, L.nb, T), dtype=torch.float32, device=L.dev)
+    ws_kept = torch.empty(cm.attn_refresh_workspace_bytes(T, h, L.kk, True), dtype=torch.uint8, device=L.dev)
+    ms_kept = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, mass,
+                                                  scale=1 / math.sqrt(d), workspace=ws_kept), 2, flush, torch)
+    aidx2 = torch.empty((h * L.nb, L.kk), dtype=torch.int32, device=L.dev)
+    ms_topk = time_events(lambda: cm.topk_cols(mass.view(h * L.nb, T), L.kk, out=aidx2), 3, flush, torch)
+    del mass, ws_kept, aidx2
     dense_attn_f = 4 * T * T * d * h
     rows["hunyuan_refresh"] = {
         "mlp_us": round(ms_mlp * 1e3, 1), "mlp_tflops": round(4 * T * D * H / (ms_mlp * 1e-3) / 1e12, 1),
-        "attn_us": round(ms_attn * 1e3, 1), "attn_passes": "dense + mass + top-k + complement",
+        "attn_us": round(ms_attn * 1e3, 1), "attn_passes": "dense + fused mass/top-k + complement",
         "attn_tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1),
-        "topk": dict(rows=h * L.nb, n=T, k=L.kk, **gbs(h * L.nb * (T + L.kk) * 4, ms_topk)),
+        "attn_us_mass_kept": round(ms_kept * 1e3, 1),
+        "mass_bytes_not_written": h * L.nb * T * 4,
+        "standalone_topk_on_kept_mass": dict(rows=h * L.nb, n=T, k=L.kk, **gbs(h * L.nb * (T + L.kk) * 4, ms_topk)),
         "us": round((ms_mlp + ms_attn) * 1e3, 1)}
 
 
@@ -708,11 +717,12 @@ def refresh_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
     ms_mlp = time_events(lambda: cm.mlp_refresh(L.x_prev, L.w1t, L.b1, L.w2, L.b2, L.a_cache, L.y_cache, L.idx,
                                                 L.mlp_scores, L.out, Bt=Bt), 5, flush, torch)
     q, k, v = L.qkv_prev
-    ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, L.mass,
-                                                  scale=1 / math.sqrt(w["d"]), workspace=L.attn_ws), 5, flush, torch)
+    ws = torch.empty(cm.attn_refresh_workspace_bytes(w["T"], w["heads"], L.kk, False), dtype=torch.uint8, device=L.dev)
+    ms_attn = time_events(lambda: cm.attn_refresh(q, k, v, L.aidx, L.m_c, L.l_c, L.acc_c, L.o, None,
+                                                  scale=1 / math.sqrt(w["d"]), workspace=ws), 5, flush, torch)
     rows["refresh_mlp"] = {"us": round(ms_mlp * 1e3, 1),
                            "tflops": round(dense_mlp_f / (ms_mlp * 1e-3) / 1e12, 1)}
-    rows["refresh_attn"] = {"us": round(ms_attn * 1e3, 1), "passes": "dense + mass + top-k + complement",
+    rows["refresh_attn"] = {"us": round(ms_attn * 1e3, 1), "passes": "dense + fused mass/top-k + complement",
                             "tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1)}
 
 
@@ -823,6 +833,55 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+PROFILE_CASES = ("attn_delta", "mass_select", "mass_kept", "mlp")
+
+
+def run_profile_case(args):
+    """Runs one kernel's workload at a size an ncu capture of many passes can hold (a few GB at most,
+    inputs larger than L2), `--steps` times, and prints what ran. Not a bench line.
+      attn_delta, mass_select, mass_kept: the HunyuanVideo attention (T = 118800, k = 8316) on 2 of
+        its 24 heads (heads are independent, so per-launch traffic scales by 12). attn_delta runs the
+        sparse step; mass_select the refresh without a mass tensor (the fused mass/top-k kernel keeps
+        the rows in its L2 row buffers), mass_kept the refresh writing the mass [h][nb][T] to HBM.
+      mlp: the sparse MLP step (mlp_up, mlp_down) of the FLUX.1-dev 2304x1280 layer (T = 12032)."""
+    import torch
+    from dynamic_column_sparse_b200 import chipmunk as cm
+    cm.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.profile_case == "mlp":
+        w = dict(FLUX, T=144 * 80 + 512, key="flux_2304x1280")
+        L = Layer(w, dev, seed=99)
+        for i in range(args.steps):
+            L.mlp_up(i)
+            L.mlp_down(i)
+        info = {"T": w["T"], "mlp_k": L.kc}
+    else:
+        w = dict(HUNYUAN, heads=2)
+        T, h, d = w["T"], w["heads"], w["d"]
+        kk, nb = k_of(T, w["attn_permille"]), (T + 127) // 128
+        g = torch.Generator(device=dev).manual_seed(5)
+        q, k, v = ((torch.randn((T, h, d), generator=g, device=dev)).to(torch.bfloat16) for _ in range(3))
+        idx = torch.empty((h, nb, kk), dtype=torch.int32, device=dev)
+        m_c, l_c = (torch.empty((h, T), dtype=torch.float32, device=dev) for _ in range(2))
+        acc_c = torch.empty((h, T, d), dtype=torch.float32, device=dev)
+        o = torch.empty((T, h, d), dtype=torch.bfloat16, device=dev)
+        keep = args.profile_case == "mass_kept"
+        mass = torch.empty((h, nb, T), dtype=torch.float32, device=dev) if keep else None
+        ws = torch.empty(cm.attn_refresh_workspace_bytes(T, h, kk, keep), dtype=torch.uint8, device=dev)
+        refresh = lambda: cm.attn_refresh(q, k, v, idx, m_c, l_c, acc_c, o, mass, scale=d ** -0.5, workspace=ws)
+        refresh()
+        for _ in range(args.steps):
+            if args.profile_case == "attn_delta":
+                cm.attn_delta(q, k, v, idx, m_c, l_c, acc_c, o, scale=d ** -0.5)
+            else:
+                refresh()
+        info = {"T": T, "heads": h, "attn_k": kk}
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    print(json.dumps({"profile_case": args.profile_case, "launches": args.steps, **info}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -833,7 +892,12 @@ def main():
     ap.add_argument("--rows", default="all",
                     help="comma list of extra row groups: " + ",".join(ROW_GROUPS) + " (default: all)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES,
+                    help="run one kernel's workload at a size for an ncu capture, --steps times (no bench line)")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

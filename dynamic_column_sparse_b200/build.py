@@ -18,8 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libchipmunk.so")
-SOURCES = ["api.cu", "noalloc.cu", "topk.cu", "cols.cu", "quant.cu", "mlp.cu", "attn.cu"]
-HEADERS = ["ptx.cuh", "kernels.cuh", "abi_internal.cuh"]
+SOURCES = ["api.cu", "noalloc.cu", "topk.cu", "cols.cu", "quant.cu", "mlp.cu", "attn.cu", "mass.cu"]
+HEADERS = ["ptx.cuh", "select.cuh", "kernels.cuh", "abi_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden", "-I" + os.path.join(ROOT, "include")]

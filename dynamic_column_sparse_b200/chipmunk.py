@@ -373,15 +373,25 @@ def attn_delta_compact(q, k, v, idx, lse_c, o_c, o, scale=None, stream=None):
     return o
 
 
-def attn_refresh(q, k, v, idx, m_c, l_c, acc_c, o, scores, scale=None, workspace=None, stream=None, lse_c=None,
+def attn_refresh_workspace_bytes(T: int, h: int, k: int, keep_mass: bool) -> int:
+    """Workspace of an attention refresh: the row log-sum-exp, plus the fused mass/top-k kernel's row
+    buffers when the mass is not kept (``scores=None``)."""
+    a = AttnArgs(T, h, 128, 128, k, 1.0)
+    return workspace_bytes(OP_REFRESH, RefreshArgs(REFRESH_ATTN, 0, MlpArgs(), a, 16 if keep_mass else None))
+
+
+def attn_refresh(q, k, v, idx, m_c, l_c, acc_c, o, scores=None, scale=None, workspace=None, stream=None, lse_c=None,
                  o_c=None):
-    """Dense attention step: o, mass scores [h][nb][T], new selection idx and the complement cache
-    (partial form m_c, l_c, acc_c; or, with lse_c and o_c given and m_c, l_c, acc_c None, the compact form)."""
+    """Dense attention step: o, new selection idx and the complement cache (partial form m_c, l_c, acc_c;
+    or, with lse_c and o_c given and m_c, l_c, acc_c None, the compact form). With ``scores`` [h][nb][T]
+    fp32 the attention mass is also written there; without it the mass stays in the workspace's row
+    buffers (the top-k is taken on it inside the mass kernel)."""
     lib = load_library()
     a = _attn_args(q, k, v, idx, m_c, l_c, acc_c, o, scale, idx.shape[2], lse_c=lse_c, o_c=o_c)
     T, h = q.shape[0], q.shape[1]
-    _need(scores, "scores", torch.float32, (h, (T + 127) // 128, T))
-    r = RefreshArgs(REFRESH_ATTN, 0, MlpArgs(), a, scores.data_ptr())
+    if scores is not None:
+        _need(scores, "scores", torch.float32, (h, (T + 127) // 128, T))
+    r = RefreshArgs(REFRESH_ATTN, 0, MlpArgs(), a, None if scores is None else scores.data_ptr())
     need = workspace_bytes(OP_REFRESH, r)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

@@ -181,6 +181,24 @@ chipmunk_status check_attn(const chipmunk_attn_args *a, bool refresh) {
   return CHIPMUNK_OK;
 }
 
+// Attention refresh scratch: the row log-sum-exp [h][T] fp32, then (when the
+// caller keeps no mass tensor) one mass row buffer per persistent CTA of the
+// fused mass/top-k kernel.
+size_t attn_refresh_lse_bytes(const chipmunk_attn_args *a) {
+  return (size_t(a->h) * size_t(a->T) * sizeof(float) + 255) & ~size_t(255);
+}
+
+size_t attn_refresh_ws(const chipmunk_refresh_args *r) {
+  const chipmunk_attn_args *a = &r->attn;
+  if (a->T < 1 || a->h < 1) return 0;
+  size_t bytes = attn_refresh_lse_bytes(a);
+  if (r->scores == nullptr) {
+    const int64_t tiles = int64_t(a->h) * ceil_div(a->T, 128);
+    bytes += size_t(cm::mass_row_buffers(tiles, a->T)) * size_t((a->T + 3) & ~int64_t(3)) * sizeof(float);
+  }
+  return bytes;
+}
+
 size_t mlp_delta_ws(const chipmunk_mlp_args *a) {
   if (a->k <= 0) return 0;
   const int64_t nb = ceil_div(a->T, a->Bt);
@@ -313,7 +331,7 @@ size_t chipmunk_workspace_bytes(int32_t op, const void *args) {
     case CHIPMUNK_OP_REFRESH: {
       if (!args) return 0;
       const chipmunk_refresh_args *r = static_cast<const chipmunk_refresh_args *>(args);
-      if (r->kind == CHIPMUNK_REFRESH_ATTN) return size_t(r->attn.h) * size_t(r->attn.T) * sizeof(float);
+      if (r->kind == CHIPMUNK_REFRESH_ATTN) return attn_refresh_ws(r);
       return 0;
     }
     default: return 0;
@@ -435,10 +453,10 @@ chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, void *ws, size_
 chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws, size_t ws_bytes,
                                        chipmunk_stream stream) {
   if (r == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "args is NULL");
-  if (r->scores == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "scores is NULL");
-  if (!aligned16(r->scores)) return fail(CHIPMUNK_ERR_ALIGNMENT, "scores is not 16-byte aligned");
+  if (r->scores != nullptr && !aligned16(r->scores)) return fail(CHIPMUNK_ERR_ALIGNMENT, "scores is not 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (r->kind == CHIPMUNK_REFRESH_MLP) {
+    if (r->scores == nullptr) return fail(CHIPMUNK_ERR_INVALID_ARG, "scores is NULL (the MLP refresh needs it)");
     const chipmunk_mlp_args *a = &r->mlp;
     CM_CHECK(check_mlp(a, true));
     int *status = nullptr;
@@ -465,7 +483,7 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
   if (r->kind == CHIPMUNK_REFRESH_ATTN) {
     const chipmunk_attn_args *a = &r->attn;
     CM_CHECK(check_attn(a, true));
-    const size_t need = size_t(a->h) * size_t(a->T) * sizeof(float);
+    const size_t need = attn_refresh_ws(r);
     if (ws == nullptr || ws_bytes < need)
       return fail(CHIPMUNK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
     if (!aligned16(ws)) return fail(CHIPMUNK_ERR_ALIGNMENT, "ws is not 16-byte aligned");
@@ -484,9 +502,11 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
                          static_cast<uint16_t *>(a->o), lse, status,
                          a->cache_format == CHIPMUNK_ATTN_CACHE_COMPACT, a->lse_c, static_cast<uint16_t *>(a->o_c)};
     CM_CUDA(cm::launch_attn(cm::kAttnDense, dense, tm_q, tm_k, tm_v, s), "attention refresh dense launch");
-    cm::MassParams mp{int(a->T), a->h, int(nb), sl2, lse, r->scores, status};
-    CM_CUDA(cm::launch_attn_mass(mp, tm_q, tm_k, s), "attention mass launch");
-    CM_CHECK(topk_impl(r->scores, int64_t(a->h) * nb, a->T, a->T, a->k, a->idx, a->k, status, s));
+    float *row_buf = r->scores != nullptr
+                         ? nullptr
+                         : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + attn_refresh_lse_bytes(a));
+    cm::MassParams mp{int(a->T), a->h, int(nb), a->k, sl2, lse, r->scores, row_buf, a->idx, status};
+    CM_CUDA(cm::launch_attn_mass_select(mp, tm_q, tm_k, s), "attention mass and top-k launch");
     CM_CUDA(cm::launch_attn(cm::kAttnComplement, dense, tm_q, tm_k, tm_v, s), "attention complement launch");
     return CHIPMUNK_OK;
   }

@@ -1,6 +1,6 @@
 // attn.cu - attention over a gathered key subset with an online-softmax merge,
 // plus the dense passes of the refresh (full attention with row log-sum-exp,
-// attention mass per query block, complement partial).
+// complement partial; the attention mass and its top-k are in mass.cu).
 //
 // Persistent CTAs walk (head, 128-query block) tiles. Q arrives once per tile
 // by a tiled TMA load; K and V stream in chunks of 128 keys through two-stage
@@ -633,133 +633,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
-// Attention mass of each key for one query block: D = K Q^T in TMEM (lane =
-// key, column = query), then each thread sums exp2(s - lse) over the block's
-// queries for its key.
-constexpr uint32_t kMQOff = 0;
-constexpr uint32_t kMKOff = 32768;        // 2 stages x 32 KB
-constexpr uint32_t kMBarOff = 98304;
-constexpr uint32_t kMLseOff = kMBarOff + 256;
-constexpr uint32_t kMSmem = 1024 + kMLseOff + 512 + 64;
-constexpr int kMassThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 column sums
-
-__global__ void __launch_bounds__(kMassThreads, 1)
-    attn_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const MassParams p) {
-  constexpr uint32_t kIdesc = idesc_bf16(128, 128, false, false);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = align_up<1024>(smem_raw);
-  uint8_t *sQ = smem + kMQOff;
-  uint8_t *sK = smem + kMKOff;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kMBarOff);
-  uint64_t *q_full = bars + 0;
-  uint64_t *k_full = bars + 1;   // [2]
-  uint64_t *k_empty = bars + 3;  // [2]
-  uint64_t *d_full = bars + 5;   // [2]
-  uint64_t *d_free = bars + 7;   // [2]
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *lse2 = reinterpret_cast<float *>(smem + kMLseOff);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (*(volatile int *)p.status != kDevOk) return;
-  // head-major: blocks that run at the same time read the same head's keys (L2 reuse)
-  const int hh = blockIdx.x / p.nb;
-  const int b = blockIdx.x % p.nb;
-  const int T = p.T;
-  const int nchunks = (T + 127) / 128;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&d_full[s], 1);
-      mbar_init(&d_free[s], 128);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
-    tmem_relinquish();
-  }
-  if (threadIdx.x < 128) {
-    const int gq = b * 128 + threadIdx.x;
-    lse2[threadIdx.x] = gq < T ? p.lse[static_cast<size_t>(hh) * T + gq] * kLog2e : INFINITY;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_2d(sQ, &tm_q, q_full, hh * 128, b * 128);
-      tma_load_2d(sQ + 16384, &tm_q, q_full, hh * 128 + 64, b * 128);
-    }
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i & 1;
-      if (!wait_warp(&k_empty[s], ((i >> 1) & 1) ^ 1, p.status, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&k_full[s], kTileBytes);
-        tma_load_2d(sK + s * kTileBytes, &tm_k, &k_full[s], hh * 128, i * 128);
-        tma_load_2d(sK + s * kTileBytes + 16384, &tm_k, &k_full[s], hh * 128 + 64, i * 128);
-      }
-      __syncwarp();
-    }
-  } else if (warp == 1) {
-    if (wait_warp(q_full, 0, p.status, abort_flag)) {
-      tc_fence_after();
-      const uint32_t q0 = smem_u32(sQ);
-      for (int i = 0; i < nchunks; ++i) {
-        const int s = i & 1;
-        if (!wait_warp(&k_full[s], (i >> 1) & 1, p.status, abort_flag)) break;
-        if (!wait_warp(&d_free[s], ((i >> 1) & 1) ^ 1, p.status, abort_flag)) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t k0 = smem_u32(sK + s * kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16(tmem + s * 128, sdesc_sw128(k0 + off, 16, 1024), sdesc_sw128(q0 + off, 16, 1024), kIdesc, kk > 0);
-          }
-          umma_commit(&k_empty[s]);
-          umma_commit(&d_full[s]);
-        }
-        __syncwarp();
-      }
-    }
-  } else {
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    float *mrow = p.mass + (static_cast<size_t>(hh) * p.nb + b) * T;
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i & 1;
-      if (!wait_warp(&d_full[s], (i >> 1) & 1, p.status, abort_flag)) break;
-      tc_fence_after();
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + s * 128 + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sum += exp2_approx(v[e] * p.scale_log2 - lse2[c * 32 + e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&d_free[s]);
-      const int key = i * 128 + r;
-      if (key < T) mrow[key] = sum;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
-}
-
 template <int MODE>
 uint32_t attn_smem(int64_t T) {
   const uint32_t mask_bytes = MODE == kAttnComplement ? ((static_cast<uint32_t>(T) + 31) / 32) * 4 : 0;
@@ -799,16 +672,6 @@ cudaError_t launch_attn(int mode, const AttnParams &p, const CUtensorMap &tm_q, 
     case kAttnComplement: return launch_attn_t<kAttnComplement>(p, tm_q, tm_k, tm_v, s);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_attn_mass(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k, cudaStream_t s) {
-  if (p.h <= 0 || p.nb <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(attn_mass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kMSmem));
-  if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.h) * p.nb;
-  attn_mass_kernel<<<static_cast<unsigned>(grid), kMassThreads, kMSmem, s>>>(tm_q, tm_k, p);
-  return cudaGetLastError();
 }
 
 }  // namespace cm

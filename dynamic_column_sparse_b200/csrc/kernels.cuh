@@ -104,16 +104,26 @@ struct AttnParams {
 cudaError_t launch_attn(int mode, const AttnParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                         const CUtensorMap &tm_v, cudaStream_t s);
 
+// Attention mass of every key per query block, mass[h][b][j] = sum over the
+// block's queries i of exp2(s_ij * scale_log2 - lse_i * log2 e), and the top k
+// keys of each mass row written to idx[h][b][0..k) (ascending, ties to the
+// lower index), in one kernel.
 struct MassParams {
-  int T, h, nb;
+  int T, h, nb, k;
   float scale_log2;
-  const float *lse;       // [h][T]
-  float *mass;            // [h][nb][T]
+  const float *lse;       // [h][T] (natural log)
+  float *mass;            // [h][nb][T], or nullptr: rows live in row_buf only
+  float *row_buf;         // [mass_row_buffers(h * nb, T)][round_up(T, 4)] when mass is nullptr
+  int32_t *idx;           // [h][nb][k]
   int *status;
 };
+// Row buffers the kernel uses for `tiles` tiles of rows of T on the current device (when the caller
+// keeps no mass tensor): one or two per persistent CTA.
+int64_t mass_row_buffers(int64_t tiles, int64_t T);
+cudaError_t launch_attn_mass_select(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                    cudaStream_t s);
+
 // One CTA waiting on a barrier nothing signals (bounded: records a timeout).
 cudaError_t launch_selftest_wait(int *status, cudaStream_t s);
-
-cudaError_t launch_attn_mass(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k, cudaStream_t s);
 
 }  // namespace cm

@@ -24,6 +24,7 @@
 // crowd into a few bins do not serialise on one shared-memory atomic each.
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "select.cuh"
 
 namespace cm {
 namespace {
@@ -36,12 +37,6 @@ constexpr int kStagedMaxN = 40960;    // 160 KB of keys in shared memory
 constexpr int kLongBins = 4096;       // first digit of the long-row path: the top 12 key bits
 constexpr int kLongCap = 12288;       // long-row candidates held in shared memory (96 KB: two CTAs per SM)
 constexpr int kSampleMaxK = 9216;     // the sampled-threshold path serves k up to 3/4 of the candidate buffer
-
-__device__ __forceinline__ uint32_t ordered_key(float f) {
-  uint32_t b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;  // -0 compares equal to +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 // Block-wide exclusive scan of a 64-bit value; also returns the block total.
 __device__ __forceinline__ uint64_t block_excl_scan(uint64_t v, uint64_t *warp_tot, uint64_t &total) {
@@ -203,18 +198,6 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkParams p) {
       __syncthreads();
     }
     row_generic<STAGED>(src, dst, n, k, staged, hist, warp_tot, s_digit, s_above);
-  }
-}
-
-// One shared-memory increment of hist[bin] for every lane that has `active`
-// set, one atomic per distinct bin of the warp (scores that crowd into a few
-// bins would otherwise serialise on them). Warp-collective: every lane of the
-// warp must call it.
-__device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
-  const unsigned am = __ballot_sync(0xffffffffu, active);
-  if (active) {
-    const unsigned peers = __match_any_sync(am, bin);
-    if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
   }
 }
 

@@ -70,11 +70,14 @@ class SparseDeltaAttention:
     ``q, k, v`` are [T][h][128] bf16. ``density_permille`` is the kept
     fraction of keys per (head, 128-query block). With ``compact`` the
     complement is cached as ``lse_c`` (fp32) and the normalised ``o_c`` (bf16)
-    instead of ``m_c``, ``l_c``, ``acc_c`` (fp32): half the bytes.
+    instead of ``m_c``, ``l_c``, ``acc_c`` (fp32): half the bytes. With
+    ``keep_mass`` the refresh also keeps the attention mass ``scores``
+    [h][nb][T] (fp32); otherwise the mass never leaves the refresh kernel's
+    row buffers.
     """
 
     def __init__(self, T: int, h: int, device, density_permille: int = 165, scale: float | None = None,
-                 compact: bool = False):
+                 compact: bool = False, keep_mass: bool = False):
         d = 128
         self.T, self.h, self.d = T, h, d
         self.nb = (T + 127) // 128
@@ -93,8 +96,9 @@ class SparseDeltaAttention:
             self.acc_c = torch.empty((h, T, d), dtype=f32, device=device)
             self.lse_c = self.o_c = None
         self.o = torch.empty((T, h, d), dtype=torch.bfloat16, device=device)
-        self.scores = torch.empty((h, self.nb, T), dtype=f32, device=device)
-        self.workspace = torch.empty(h * T * 4, dtype=torch.uint8, device=device)
+        self.scores = torch.empty((h, self.nb, T), dtype=f32, device=device) if keep_mass else None
+        self.workspace = torch.empty(cm.attn_refresh_workspace_bytes(T, h, self.k, keep_mass), dtype=torch.uint8,
+                                     device=device)
         self.has_cache = False
 
     def refresh(self, q, k, v, stream=None):

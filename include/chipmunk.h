@@ -156,11 +156,16 @@ typedef struct chipmunk_attn_args {
  *     is non-zero), mlp.idx (top mlp.k columns of each score row),
  *     mlp.a_cache = bf16(a), mlp.y_cache = a W2 + b2 and mlp.out (if not NULL).
  *   kind == CHIPMUNK_REFRESH_ATTN: reads attn.{q,kk,v}; writes attn.o (dense
- *     attention), scores [h][nb][T] (fp32 attention mass: per query block
- *     the column sums of the softmax probabilities), attn.idx (top attn.k keys
- *     of each mass row) and the complement cache of every query over the
- *     keys its block did not select, in attn.cache_format: attn.{m_c,l_c,acc_c}
- *     or attn.{lse_c,o_c}.
+ *     attention), attn.idx (top attn.k keys of each row of the attention
+ *     mass: per head and query block the column sums of the softmax
+ *     probabilities, fp32; the top-k is taken inside the kernel that computes
+ *     the mass), the complement cache of every query over the keys its block
+ *     did not select, in attn.cache_format: attn.{m_c,l_c,acc_c} or
+ *     attn.{lse_c,o_c}; and, if scores is not NULL, the mass itself to
+ *     scores [h][nb][T]. With scores NULL the mass rows live only in the
+ *     workspace's row buffers (the post's "fast sparsity identification":
+ *     the 4-byte-per-key mass need not travel to HBM and back).
+ * scores: 16-byte aligned; required for the MLP, optional for attention.
  */
 typedef struct chipmunk_refresh_args {
   int32_t kind;
@@ -324,8 +329,12 @@ CHIPMUNK_API chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, vo
 
 /*
  * Dense refresh (see chipmunk_refresh_args). Workspace:
- * chipmunk_workspace_bytes(CHIPMUNK_OP_REFRESH, a) bytes (attention: the row
- * log-sum-exp, h * T fp32; MLP: none).
+ * chipmunk_workspace_bytes(CHIPMUNK_OP_REFRESH, a) bytes, 16-byte aligned
+ * (MLP: none; attention: the row log-sum-exp, h * T fp32 rounded up to 256
+ * bytes, then, when a->scores is NULL, the mass kernel's row buffers: one or
+ * two rows of round_up(T, 4) fp32 per persistent CTA, sized for the current
+ * device, so query the size on the device that runs the call). Too small a
+ * workspace is rejected with CHIPMUNK_ERR_WORKSPACE before anything runs.
  */
 CHIPMUNK_API chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *a, void *ws, size_t ws_bytes,
                                        chipmunk_stream stream);

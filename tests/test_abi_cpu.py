@@ -127,8 +127,36 @@ def test_refresh_rejects_unknown_kind(cm):
     lib = cm.load_library()
     r = cm.RefreshArgs(kind=7, scores=0x1000)
     assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1
+    r = cm.RefreshArgs(kind=cm.REFRESH_MLP, scores=0)
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == cm.ERR_INVALID_ARG  # the MLP needs scores
     r = cm.RefreshArgs(kind=cm.REFRESH_ATTN, scores=0)
-    assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == 1
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), None, 0, None) == cm.ERR_SHAPE        # T = 0
+
+
+def _attn_refresh_args(cm, T, h, k, scores):
+    p = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(8)]
+    a = cm.AttnArgs(T, h, 128, 128, k, 0.088, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7])
+    return cm.RefreshArgs(cm.REFRESH_ATTN, 0, cm.MlpArgs(), a, scores)
+
+
+def test_attn_refresh_workspace_without_a_mass_tensor(cm):
+    """Without a mass tensor the refresh needs the row log-sum-exp plus the fused mass/top-k kernel's row
+    buffers (at least one row of round_up(T, 4) fp32); with one, the log-sum-exp only. Too small a
+    workspace is rejected on the host."""
+    lib = cm.load_library()
+    T, h, k = 1001, 3, 165
+    kept = cm.workspace_bytes(cm.OP_REFRESH, _attn_refresh_args(cm, T, h, k, 0x20000000))
+    fused = cm.workspace_bytes(cm.OP_REFRESH, _attn_refresh_args(cm, T, h, k, None))
+    assert kept == (h * T * 4 + 255) // 256 * 256
+    rows = (fused - kept) // (((T + 3) // 4) * 16)
+    assert fused - kept == rows * ((T + 3) // 4) * 16 and 1 <= rows <= h * ((T + 127) // 128)
+    assert cm.attn_refresh_workspace_bytes(T, h, k, False) == fused
+    assert cm.attn_refresh_workspace_bytes(T, h, k, True) == kept
+    r = _attn_refresh_args(cm, T, h, k, None)
+    ws = ctypes.c_void_p(0x40000000)
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), ws, fused - 16, None) == cm.ERR_WORKSPACE
+    r = _attn_refresh_args(cm, T, h, k, 0x20000004)
+    assert lib.chipmunk_dense_refresh(ctypes.byref(r), ws, kept, None) == cm.ERR_ALIGNMENT   # scores misaligned
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch(cm):

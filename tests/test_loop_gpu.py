@@ -119,7 +119,7 @@ def run_attn_loop(T, h, permille, seed=4):
     from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaAttention
     chains = {n: drift_chain(synth.normal_bf16(seed, synth.TID[n + "_prev"], (T, h, 128)), seed,
                              synth.TID[n + "_drift"], 0.03, STEPS) for n in ("q", "k", "v")}
-    layer = SparseDeltaAttention(T, h, "cuda", permille)
+    layer = SparseDeltaAttention(T, h, "cuda", permille, keep_mass=True)
     sched = Schedule(DENSE_STEPS)
     scale = 1.0 / math.sqrt(128)
     kk = O.k_from_density(T, permille)

@@ -10,7 +10,7 @@ import pytest
 
 import oracle as O
 from dynamic_column_sparse_b200 import synth
-from helpers import (assert_bf16_storage, check_selection, assert_parity, bits_of, dev_bf16, dev_f32, f64_of, f64_of_bf16, heads_first, to_block_major,
+from helpers import (assert_bf16_storage, assert_is_topk_of, check_selection, assert_parity, bits_of, dev_bf16, dev_f32, f64_of, f64_of_bf16, heads_first, to_block_major,
                      to_token_major)
 
 pytestmark = pytest.mark.gpu
@@ -79,6 +79,7 @@ def test_attn_refresh(cm, T, h, permille):
     assert_parity(heads_first(f64_of_bf16(o)), ref["O"], "o", bf16_out=True)
     assert_parity(f64_of(scores), ref["mass"], "mass", max_of_rms=5e-3, mean_rel=1e-3)
     g_idx = idx.cpu().numpy()
+    assert_is_topk_of(g_idx.reshape(h * nb, kk), scores.cpu().numpy().reshape(h * nb, T), "selection vs its own mass")
     same = check_selection(g_idx.reshape(h * nb, kk), ref["mass"].reshape(h * nb, T), kk, band=2e-3)
     assert same >= 0.9 * h * nb
     # complement cache on rows whose selection matches the oracle's

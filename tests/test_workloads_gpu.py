@@ -247,9 +247,10 @@ def test_mlp_refresh_sampled_hunyuan():
 
 
 def test_attention_refresh_sampled_hunyuan():
-    """Dense attention refresh at T = 118800 (dense pass, attention mass, top-k over 22296 rows of
-    118800, complement pass): output, mass rows, selection and complement cache on 32 sampled
-    (head, query-block) tiles."""
+    """Dense attention refresh at T = 118800 (dense pass, attention mass with the top-k over its 22296
+    rows of 118800, complement pass): output, mass rows, selection and complement cache on 32 sampled
+    (head, query-block) tiles; every row's selection against the standalone top-k of the kept mass;
+    the refresh without a mass tensor against the one with."""
     import torch
     from dynamic_column_sparse_b200 import chipmunk as cm
     T = 118800
@@ -321,3 +322,15 @@ def test_attention_refresh_sampled_hunyuan():
     assert got_c, "no sampled tile selects as the oracle does"
     assert_parity(np.concatenate(got_c), np.concatenate(ref_c), "complement acc/l (matching tiles)")
     assert np.max(np.abs(np.concatenate(got_lse) - np.concatenate(ref_lse))) < 1e-3, "complement log-sum-exp"
+    # every row's in-kernel selection equals the standalone top-k kernel's on the same kept mass rows
+    # (that kernel is bit-exact against the oracle's top-k in the top-k tests)
+    alone = cm.topk_cols(mass.view(NH * NB, T), kk)
+    assert torch.equal(alone, layer_idx.view(NH * NB, kk)), "fused selection vs standalone top-k"
+    # without a mass tensor the mass stays in the kernel's row buffers: the same selection, output and cache
+    del mass, alone
+    kept = [t.clone() for t in (layer_idx, o, m_c, l_c, acc_c)]
+    cm.attn_refresh(q, kt, vt, layer_idx, m_c, l_c, acc_c, o, None, scale=scale)
+    torch.cuda.synchronize()
+    assert cm.read_device_status() == 0
+    for a, b, what in zip((layer_idx, o, m_c, l_c, acc_c), kept, ("idx", "o", "m_c", "l_c", "acc_c")):
+        assert torch.equal(a, b), f"refresh without a mass tensor: {what} differs"
