@@ -194,7 +194,8 @@ size_t attn_refresh_ws(const chipmunk_refresh_args *r) {
   size_t bytes = attn_refresh_lse_bytes(a);
   if (r->scores == nullptr) {
     const int64_t tiles = int64_t(a->h) * ceil_div(a->T, 128);
-    bytes += size_t(cm::mass_row_buffers(tiles, a->T)) * size_t((a->T + 3) & ~int64_t(3)) * sizeof(float);
+    // + 128: the row buffers start at the first 128-byte boundary after the log-sum-exp
+    bytes += 128 + size_t(cm::mass_row_buffers(tiles, a->T)) * size_t(cm::mass_row_floats(a->T)) * sizeof(float);
   }
   return bytes;
 }
@@ -502,9 +503,8 @@ chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *r, void *ws,
                          static_cast<uint16_t *>(a->o), lse, status,
                          a->cache_format == CHIPMUNK_ATTN_CACHE_COMPACT, a->lse_c, static_cast<uint16_t *>(a->o_c)};
     CM_CUDA(cm::launch_attn(cm::kAttnDense, dense, tm_q, tm_k, tm_v, s), "attention refresh dense launch");
-    float *row_buf = r->scores != nullptr
-                         ? nullptr
-                         : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + attn_refresh_lse_bytes(a));
+    const uintptr_t rows_at = (reinterpret_cast<uintptr_t>(ws) + attn_refresh_lse_bytes(a) + 127) & ~uintptr_t(127);
+    float *row_buf = r->scores != nullptr ? nullptr : reinterpret_cast<float *>(rows_at);
     cm::MassParams mp{int(a->T), a->h, int(nb), a->k, sl2, lse, r->scores, row_buf, a->idx, status};
     CM_CUDA(cm::launch_attn_mass_select(mp, tm_q, tm_k, s), "attention mass and top-k launch");
     CM_CUDA(cm::launch_attn(cm::kAttnComplement, dense, tm_q, tm_k, tm_v, s), "attention complement launch");

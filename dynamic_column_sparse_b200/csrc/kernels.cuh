@@ -113,13 +113,14 @@ struct MassParams {
   float scale_log2;
   const float *lse;       // [h][T] (natural log)
   float *mass;            // [h][nb][T], or nullptr: rows live in row_buf only
-  float *row_buf;         // [mass_row_buffers(h * nb, T)][round_up(T, 4)] when mass is nullptr
+  float *row_buf;         // [mass_row_buffers(h * nb, T)][mass_row_floats(T)], 128-byte aligned, when mass is nullptr
   int32_t *idx;           // [h][nb][k]
   int *status;
 };
 // Row buffers the kernel uses for `tiles` tiles of rows of T on the current device (when the caller
 // keeps no mass tensor): one or two per persistent CTA.
 int64_t mass_row_buffers(int64_t tiles, int64_t T);
+int64_t mass_row_floats(int64_t T);
 cudaError_t launch_attn_mass_select(const MassParams &p, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                     cudaStream_t s);
 

@@ -62,10 +62,12 @@ constexpr uint32_t kSelOff = kCIdxOff + kCap * 4;        // scan words, digit re
 constexpr uint32_t kSmem = 1024 + kSelOff + 256;
 static_assert(kSmem <= 232448, "shared memory of one CTA");
 
+// Floats per row buffer: whole 128-byte lines, so that a row's lines hold no other row.
+__host__ __device__ __forceinline__ int64_t mass_row_pad(int64_t T) { return (T + 31) & ~static_cast<int64_t>(31); }
+
 // Row buffers per CTA: two when those of all `grid` CTAs fit in kTwoSlotBytes.
 __host__ __device__ __forceinline__ int64_t mass_row_slots(int64_t grid, int64_t T) {
-  const int64_t row_bytes = ((T + 3) & ~static_cast<int64_t>(3)) * 4;
-  return 2 * grid * row_bytes <= kTwoSlotBytes ? 2 : 1;
+  return 2 * grid * mass_row_pad(T) * 4 <= kTwoSlotBytes ? 2 : 1;
 }
 
 __device__ __forceinline__ uint32_t mass_bin(uint32_t key) {
@@ -86,6 +88,22 @@ __device__ __forceinline__ uint64_t ld_acquire_shared(const uint64_t *p) {
 
 __device__ __forceinline__ void st_release_shared(uint64_t *p, uint64_t v) {
   asm volatile("st.release.cta.shared::cta.u64 [%0], %1;" ::"r"(smem_u32(p)), "l"(v) : "memory");
+}
+
+// An L2 policy that evicts the lines it touches after others (the live mass rows).
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void st_global_hint(float *p, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
+// Drops the 128-byte line at p from L2 without writing it back (its data is dead).
+__device__ __forceinline__ void discard_l2_line(const void *p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
@@ -160,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nch = (T + 127) / 128;
   const int tiles = p.h * p.nb;
   const bool shared_row = p.mass == nullptr;
-  const int64_t row_pad = (static_cast<int64_t>(T) + 3) & ~static_cast<int64_t>(3);
+  const int64_t row_pad = mass_row_pad(T);
   const int slots = static_cast<int>(mass_row_slots(gridDim.x, T));
   // the mass row of local tile j (global tile t)
   auto row_of = [&](int j, int t) -> float * {
@@ -272,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     uint32_t g = 0;
     uint64_t seen = 0;
+    const uint64_t pol = l2_evict_last_policy();
     for (int j = 0, t = blockIdx.x; t < tiles; ++j, t += gridDim.x) {
       if (!wait_warp(&lse_full[j & 1], (j >> 1) & 1, p.status, abort_flag)) break;
       if (!wait_warp(&hist_free[j & 1], ((j >> 1) & 1) ^ 1, p.status, abort_flag)) break;
@@ -305,7 +324,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (key < T) row[key] = sum;
+        if (key < T) {
+          if (shared_row) {
+            st_global_hint(row + key, sum, pol);
+          } else {
+            row[key] = sum;
+          }
+        }
         warp_hist_add(hcur, mass_bin(ordered_key(sum)), key < T);
       }
       if (!ok) break;
@@ -323,12 +348,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t *dst = p.idx + static_cast<size_t>(t) * k;
       uint32_t *hrow = hist + (j & 1) * kBins;
       const uint64_t done_before = static_cast<uint64_t>(j) * nch;
-      // publishes that the first `end` elements of this row have been read
+      int read_end = 0;  // elements of a row buffer already read and released
+      // Group-wide, after the first `end` elements of the row have been read for the last time: in a
+      // row buffer, drops their lines from L2 (dead data is never written back) and publishes the
+      // progress that lets the mass warps overwrite them.
       auto tile_done = [&](int end) {
-        if (st == 0 && shared_row) {
+        end = min(end, T);
+        if (!shared_row || end <= read_end) return;
+        const int64_t l1 = (static_cast<int64_t>(end) + 31) / 32;
+        for (int64_t l = read_end / 32 + st; l < l1; l += kSelThreads) discard_l2_line(row + l * 32);
+        Sel::sync();
+        if (st == 0) {
           const uint64_t c = end >= T ? static_cast<uint64_t>(nch) : static_cast<uint64_t>(end / 128);
           st_release_shared(progress, done_before + c);
         }
+        read_end = end;
       };
       if (k >= T) {
         for (int i = st; i < T; i += kSelThreads) dst[i] = i;
@@ -409,6 +443,8 @@ int64_t mass_grid(int64_t tiles) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return std::min<int64_t>(tiles, std::max(sms, 1));
 }
+
+int64_t mass_row_floats(int64_t T) { return mass_row_pad(T); }
 
 int64_t mass_row_buffers(int64_t tiles, int64_t T) {
   const int64_t grid = mass_grid(tiles);

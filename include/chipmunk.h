@@ -331,9 +331,10 @@ CHIPMUNK_API chipmunk_status chipmunk_attn_delta(const chipmunk_attn_args *a, vo
  * Dense refresh (see chipmunk_refresh_args). Workspace:
  * chipmunk_workspace_bytes(CHIPMUNK_OP_REFRESH, a) bytes, 16-byte aligned
  * (MLP: none; attention: the row log-sum-exp, h * T fp32 rounded up to 256
- * bytes, then, when a->scores is NULL, the mass kernel's row buffers: one or
- * two rows of round_up(T, 4) fp32 per persistent CTA, sized for the current
- * device, so query the size on the device that runs the call). Too small a
+ * bytes, then, when a->scores is NULL, the mass kernel's row buffers from the
+ * next 128-byte boundary: one or two rows of round_up(T, 32) fp32 per
+ * persistent CTA, sized for the current device, so query the size on the
+ * device that runs the call). Too small a
  * workspace is rejected with CHIPMUNK_ERR_WORKSPACE before anything runs.
  */
 CHIPMUNK_API chipmunk_status chipmunk_dense_refresh(const chipmunk_refresh_args *a, void *ws, size_t ws_bytes,

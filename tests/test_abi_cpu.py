@@ -141,15 +141,16 @@ def _attn_refresh_args(cm, T, h, k, scores):
 
 def test_attn_refresh_workspace_without_a_mass_tensor(cm):
     """Without a mass tensor the refresh needs the row log-sum-exp plus the fused mass/top-k kernel's row
-    buffers (at least one row of round_up(T, 4) fp32); with one, the log-sum-exp only. Too small a
-    workspace is rejected on the host."""
+    buffers (at least one row of round_up(T, 32) fp32, from a 128-byte boundary); with one, the
+    log-sum-exp only. Too small a workspace is rejected on the host."""
     lib = cm.load_library()
     T, h, k = 1001, 3, 165
     kept = cm.workspace_bytes(cm.OP_REFRESH, _attn_refresh_args(cm, T, h, k, 0x20000000))
     fused = cm.workspace_bytes(cm.OP_REFRESH, _attn_refresh_args(cm, T, h, k, None))
     assert kept == (h * T * 4 + 255) // 256 * 256
-    rows = (fused - kept) // (((T + 3) // 4) * 16)
-    assert fused - kept == rows * ((T + 3) // 4) * 16 and 1 <= rows <= h * ((T + 127) // 128)
+    row_bytes = (T + 31) // 32 * 128
+    rows = (fused - kept - 128) // row_bytes
+    assert fused - kept == 128 + rows * row_bytes and 1 <= rows <= h * ((T + 127) // 128)
     assert cm.attn_refresh_workspace_bytes(T, h, k, False) == fused
     assert cm.attn_refresh_workspace_bytes(T, h, k, True) == kept
     r = _attn_refresh_args(cm, T, h, k, None)
