@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *mask_bar = bars + 25;  // softmax warps: complement mask steps
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint64_t *qt_full = bars + 27;   // [2] Q of a tile is in TMEM buffer tile & 1
+  uint64_t *qt_empty = bars + 29;  // [2] the last S = Q K^T of the tile two back has read that buffer
   int *kidx = reinterpret_cast<int *>(smem + C::kIdxOff);        // [4][128] selected keys of chunk g at g & 3
   float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);   // [2][2][128] partial row sums
   float *xmax = reinterpret_cast<float *>(smem + C::kXmaxOff);   // [2][2][128] partial row maxima by chunk parity
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, kSoftmaxThreads);   // the softmax warps have copied Q into TMEM
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], MODE == kAttnDelta ? kProducers : 1);
       mbar_init(&v_full[s], MODE == kAttnDelta ? kProducers : 1);
@@ -115,6 +117,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(o_full, 1);
     mbar_init(o_empty, kSoftmaxThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qt_full[s], kSoftmaxThreads);
+      mbar_init(&qt_empty[s], 1);
+    }
     for (int qd = 0; qd < 4; ++qd) mbar_init(&pair_bar[qd], 64);
     mbar_init(mask_bar, kSoftmaxThreads);
     *abort_flag = 0;
@@ -132,7 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S[0] at column 0, S[1] at 128, O at 256, P[0] at 384, P[1] at 448
+  // TMEM columns: S[0] at 0, S[1] at 128 (P of a chunk, bf16 pairs, overwrites the first 64 columns of
+  // its S buffer), O at 256, Q[0] at 384, Q[1] at 448 (bf16 pairs: the A operand of S = Q K^T)
+  const uint32_t tmem = *tmem_slot;
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ producers
@@ -142,7 +150,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ahead of V; the last V of a tile goes out before the next tile's loads.
     // g counts chunks over this CTA's tiles.
     const int pw = warp - kProdWarp0;
-    const int pt = threadIdx.x - kProdWarp0 * 32;  // 0..223
     const int my_tiles = static_cast<int>(blockIdx.x) < ntiles ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
     const int total = my_tiles * nchunks;
     // warp pw moves rows 20 pw .. 20 pw + 19 (< 128) of every chunk and
@@ -258,10 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     int tl = 0;
     bool ok = true;
-    const uint32_t q0 = smem_u32(sQ);
     const uint32_t tO = tmem + 256;
     for (int tile = blockIdx.x; tile < ntiles && ok && nchunks > 0; tile += gridDim.x, ++tl) {
-      if (!wait_warp(q_full, tl & 1, p.status, abort_flag)) break;
+      if (!wait_warp(&qt_full[tl & 1], (tl >> 1) & 1, p.status, abort_flag)) break;
+      const uint32_t tQ = tmem + 384 + (tl & 1) * 64;
       for (int i = 0; i <= nchunks && ok; ++i) {
         if (i < nchunks) {
           const int g = tl * nchunks + i, s = g & 1;
@@ -277,12 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              umma_bf16(tmem + s * 128, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(k0 + off, 16, 1024), kIdescQK,
-                        kk > 0);
+              umma_bf16_ts(tmem + s * 128, tQ + kk * 8, sdesc_sw128(k0 + off, 16, 1024), kIdescQK, kk > 0);
             }
             umma_commit(&s_full[s]);
             umma_commit(&k_empty[s]);
-            if (i == nchunks - 1) umma_commit(q_empty);
+            if (i == nchunks - 1) umma_commit(&qt_empty[tl & 1]);
           }
           __syncwarp();
         }
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t v0 = smem_u32(sV + s * kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_bf16_ts(tO, tmem + 384 + s * 64 + kk * 8, sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV,
+              umma_bf16_ts(tO, tmem + s * 128 + kk * 8, sdesc_sw128(v0 + kk * 2048, 16384, 1024), kIdescPV,
                            (j | kk) != 0);
             umma_commit(&v_empty[s]);
             umma_commit(&p_empty[s]);
@@ -337,8 +343,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++mask_phase;
       return r2;
     };
+    // Q of this CTA's tile tq (arrived by TMA in shared memory) into TMEM buffer tq & 1: this
+    // thread's row r, dimensions 64 half .. 64 half + 63 as 32 columns of bf16 pairs; then the
+    // shared-memory tile is free for the next tile's Q
+    auto copy_q = [&](int tq) -> bool {
+      if (!wait_warp(q_full, tq & 1, p.status, abort_flag) ||
+          !wait_warp(&qt_empty[tq & 1], ((tq >> 1) & 1) ^ 1, p.status, abort_flag))
+        return false;
+      tc_fence_after();
+      uint32_t wq[32];
+      const uint8_t *qh = sQ + half * 16384;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(qh + sw128_offset(r, c));
+        wq[4 * c] = u.x, wq[4 * c + 1] = u.y, wq[4 * c + 2] = u.z, wq[4 * c + 3] = u.w;
+      }
+      tmem_st32(tmem + lane_off + 384 + (tq & 1) * 64 + half * 32, reinterpret_cast<const float *>(wq));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&qt_full[tq & 1]);
+      mbar_arrive(q_empty);
+      return true;
+    };
     int tl = 0;
     bool ok = true;
+    if (nchunks > 0 && static_cast<int>(blockIdx.x) < ntiles && !copy_q(0)) ok = false;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tl) {
       const int hh = tile / p.nb, b = tile % p.nb;
       const int gi = b * 128 + r;
@@ -454,21 +483,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           lp[e & 3] += sv[e];
         }
         l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-        // P into TMEM buffer g & 1 (this row's keys 64h .. 64h+63 as 32 columns of
-        // bf16 pairs), once P V of chunk g - 2 has read that buffer
-        if (!wait_warp(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, p.status, abort_flag)) {
-          ok = false;
-          break;
-        }
+        // P over the first 64 columns of S buffer g & 1 (this row's keys 64h .. 64h+63 as 32
+        // columns of bf16 pairs). Both warps of the quadrant have read their half of S (the
+        // exchange above), and P V of chunk g - 2, which read the buffer's previous P, was issued
+        // before S = Q K^T of chunk g wrote it (tensor-core operations run in issue order).
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = cvt_bf16x2(sv[2 * e], sv[2 * e + 1]);
-        tmem_st32(tmem + lane_off + 384 + (g & 1) * 64 + half * 32, reinterpret_cast<const float *>(pk));
+        tc_fence_after();
+        tmem_st32(tmem + lane_off + (g & 1) * 128 + half * 32, reinterpret_cast<const float *>(pk));
         tmem_wait_st();
         tc_fence_before();  // orders the P stores (and a rescale's O stores) before the next P V
         mbar_arrive(&p_full[g & 1]);
       }
       if (!ok) break;
+      // the next tile's Q into TMEM now, so its first S = Q K^T overlaps this tile's epilogue
+      if (nchunks > 0 && tile + static_cast<int>(gridDim.x) < ntiles && !copy_q(tl + 1)) break;
       // row sum over both halves (buffer by tile parity: the next write to it is two tiles away)
       float *xs = xsum + ob * 256;
       xs[half * 128 + r] = l;
