@@ -619,19 +619,15 @@ def extra_rows(L, w, peaks, flush, torch, cm, groups=frozenset(ROW_GROUPS)):
     dense_attn_f = 4 * T * T * wf["d"] * h
     if "refresh" in groups:
         refresh_rows(LF, wf, rows, flush, torch, cm, dense_mlp_f, dense_attn_f)
+    lib_dense_us = None
+    if "cublas" in groups:
+        lib_dense_us = library_dense_rows(LF, wf, rows, flush, torch)
     if "dense" in groups or "sweep" in groups:
         dense_us = dense_rows(LF, wf, rows, flush, torch, cm, dense_mlp_f, dense_attn_f)
         if "sweep" in groups:
-            sweep_rows(LF, wf, rows, flush, torch, dense_us)
+            sweep_rows(LF, wf, rows, flush, torch, dense_us, lib_dense_us)
     if "compact" in groups:
         compact_rows(LF, wf, rows, flush, torch, hbm)
-    if "cublas" in groups:
-        xw = LF.xs[0]
-        w1 = LF.w1t.t()
-        ms_cub = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),
-                                                  LF.w2), 5, flush, torch)
-        rows["dense_mlp_torch_context"] = {"us": round(ms_cub * 1e3, 1), "T": T,
-                                           "note": "torch.matmul (cuBLAS) + GELU at the FLUX 1280x768 shape, context only"}
     del LF
     torch.cuda.synchronize()
     assert cm.read_device_status() == 0
@@ -746,6 +742,24 @@ def dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
     return (ms_dm + ms_da) * 1e3
 
 
+def library_dense_rows(L, w, rows, flush, torch):
+    """Context only: the dense FLUX layer with library kernels, torch.matmul (cuBLAS) + GELU for the MLP and
+    torch's scaled_dot_product_attention for the attention. Returns the layer's us."""
+    T, h, d = w["T"], w["heads"], w["d"]
+    xw, w1 = L.xs[0], L.w1t.t()
+    ms_mlp = time_events(lambda: torch.matmul(torch.nn.functional.gelu(torch.matmul(xw, w1), approximate="tanh"),
+                                              L.w2), 5, flush, torch)
+    q, k, v = (t.view(1, T, h, d).transpose(1, 2) for t in L.qkvs[0])
+    ms_attn = time_events(lambda: torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=d ** -0.5), 5,
+                          flush, torch)
+    rows["dense_mlp_torch_context"] = {"us": round(ms_mlp * 1e3, 1), "T": T,
+                                       "note": "torch.matmul (cuBLAS) + GELU at the FLUX 1280x768 shape, context only"}
+    rows["dense_attn_torch_sdpa_context"] = {"us": round(ms_attn * 1e3, 1), "T": T, "heads": h,
+                                             "note": "torch scaled_dot_product_attention at the FLUX 1280x768 shape, "
+                                                     "context only"}
+    return (ms_mlp + ms_attn) * 1e3
+
+
 def compact_rows(L, w, rows, flush, torch, hbm):
     """Attention delta step with the complement cached as fp32 (m, l, acc) or compact (lse fp32, o_c bf16)."""
     from dynamic_column_sparse_b200.layer import SparseDeltaAttention
@@ -770,8 +784,10 @@ def compact_rows(L, w, rows, flush, torch, hbm):
     rows["attn_delta_cache_forms"] = out
 
 
-def sweep_rows(L, w, rows, flush, torch, dense_us):
-    """Multi-step schedule (10 steps, dense at 0 and 5) across sparsity levels, through the layer API."""
+def sweep_rows(L, w, rows, flush, torch, dense_us, lib_dense_us=None):
+    """Multi-step schedule (10 steps, dense at 0 and 5) across sparsity levels, through the layer API.
+    The speed-ups are against this library's own dense layer (k = all) and, when timed, against the
+    faster of that and the library-kernel dense layer (cuBLAS MLP + torch attention)."""
     from dynamic_column_sparse_b200.layer import Schedule, SparseDeltaAttention, SparseDeltaMLP
     T, h, Bt = w["T"], w["heads"], w["Bt"]
     reps = 10
@@ -796,6 +812,11 @@ def sweep_rows(L, w, rows, flush, torch, dense_us):
             "mlp_k": mlp.k, "attn_k": att.k, "sparse_step_us": round(ms_sp * 1e3, 1),
             "refresh_us": round(ms_ref * 1e3, 1), "loop10_us_per_layer_step": round(amort, 1),
             "speedup_vs_dense_k_all": round(dense_us / (ms_sp * 1e3), 2)}
+        if lib_dense_us is not None:
+            best = min(dense_us, lib_dense_us)
+            sweep[f"mlp{100 - mp // 10}_attn{round(100 - ap / 10, 1)}"].update(
+                speedup_vs_fastest_dense=round(best / (ms_sp * 1e3), 2),
+                loop10_speedup_vs_fastest_dense=round(best / amort, 2))
         del mlp, att
     rows["loop_sweep"] = sweep
 
