@@ -655,7 +655,7 @@ def hunyuan_refresh_rows(L, w, rows, gbs, flush, torch, cm):
     rows["hunyuan_refresh"] = {
         "mlp_us": round(ms_mlp * 1e3, 1), "mlp_tflops": round(4 * T * D * H / (ms_mlp * 1e-3) / 1e12, 1),
         "attn_us": round(ms_attn * 1e3, 1), "attn_passes": "dense + fused mass/top-k + complement",
-        "attn_tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1),
+        "attn_tflops_mma": round(2.5 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1),
         "attn_us_mass_kept": round(ms_kept * 1e3, 1),
         "mass_bytes_not_written": h * L.nb * T * 4,
         "standalone_topk_on_kept_mass": dict(rows=h * L.nb, n=T, k=L.kk, **gbs(h * L.nb * (T + L.kk) * 4, ms_topk)),
@@ -719,7 +719,7 @@ def refresh_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):
     rows["refresh_mlp"] = {"us": round(ms_mlp * 1e3, 1),
                            "tflops": round(dense_mlp_f / (ms_mlp * 1e-3) / 1e12, 1)}
     rows["refresh_attn"] = {"us": round(ms_attn * 1e3, 1), "passes": "dense + fused mass/top-k + complement",
-                            "tflops_3_passes": round(3 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1)}
+                            "tflops_mma": round(2.5 * dense_attn_f / (ms_attn * 1e-3) / 1e12, 1)}
 
 
 def dense_rows(L, w, rows, flush, torch, cm, dense_mlp_f, dense_attn_f):

@@ -45,6 +45,7 @@ struct MlpUpParams {
   // FP8 step only: x ~ sx[t] * x8[t][:], W1^T ~ s1[c] * w1t8[c][:], the delta
   // of column c is multiplied by g2[c] before it is rounded to e4m3
   const float *sx, *s1, *g2;
+  int group;              // token blocks walked together (set by the launcher)
 };
 // tm_w1t: tile map over W1^T [H][D] (box 64 x 128), read on a refresh only.
 cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s);
@@ -67,6 +68,7 @@ struct MlpDownParams {
   uint16_t *out;          // [T][D] or nullptr
   int *status;
   float s_delta;          // FP8 step only: the scale of the delta codes
+  int group;              // token blocks walked together (set by the launcher)
 };
 // tm_a: 3-D map over A [nb][rows][Bt]; tm_w2: tile map over W2 [H][D] (box 64 x 64), read on a refresh only.
 cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,

@@ -57,6 +57,42 @@ struct Roles {
 
 constexpr int kBK = 64;  // K elements per pipeline stage = one 128-byte swizzle row
 
+// The order in which a CTA's tiles are walked. Tile t of nb token blocks x
+// nparts parts of a block (chunks of its selected columns, or slices of the
+// output) is taken a group of `group` blocks at a time, part-major inside the
+// group: CTAs running at the same time work on the same part of different
+// blocks, so they gather weight rows from the same region of the (ascending)
+// index lists, and a group's activation tiles stay in L2 until all of its
+// parts are done instead of being read from HBM again for every part. With
+// group = nb this is part-major over the whole layer.
+struct TileAt {
+  int b, part;
+};
+
+__device__ __forceinline__ TileAt tile_at(int t, int nb, int nparts, int group) {
+  const int per_group = group * nparts;
+  const int g = t / per_group, r = t - g * per_group;
+  const int b0 = g * group;
+  const int gb = min(group, nb - b0);   // blocks in this group (the last may be short)
+  return {b0 + r % gb, r / gb};
+}
+
+// Blocks walked together: all of them when the layer's activation tiles (x for
+// the up-projection) fit in well under half of L2 (the FLUX.1-dev 1280x768 layer), else
+// as many as fill about 24 MB (32 blocks of 128 tokens at D = 3072 in bf16).
+int up_tile_group(int nb, int64_t tile_bytes) {
+  if (static_cast<int64_t>(nb) * tile_bytes <= (48ll << 20)) return nb;
+  return std::max<int>(8, static_cast<int>((24ll << 20) / tile_bytes));
+}
+
+// The sparse down-projection walks slice-major over all blocks: every CTA
+// running at a time gathers W2 rows of the same output slice, which matters
+// more for it than keeping the delta tiles of a group in L2 (measured). The
+// dense one (a refresh) reads every block's whole activation-cache tile (3 MB at
+// H = 12288) once per output slice, so it is walked in groups like the
+// up-projection.
+int down_tile_group(int nb, bool dense, int64_t tile_bytes) { return dense ? up_tile_group(nb, tile_bytes) : nb; }
+
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag) {
   const bool ok = mbar_wait(bar, parity, status, abort_flag);
@@ -79,9 +115,10 @@ struct UpCfg : Roles<4, 4> {
   static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "two CTAs must fit in one SM's shared memory");
 };
 
-// Persistent: CTA c handles tiles c, c + gridDim.x, ... where tile = chunk * nb
-// + b (chunk-major: index lists are ascending, so CTAs running at the same
-// time gather W1^T rows from the same region, for L2 reuse). Two TMEM
+// Persistent: CTA c handles tiles c, c + gridDim.x, ..., tile t being chunk
+// tile_at(t).part of block tile_at(t).b (grouped, chunk-major in a group: CTAs
+// running at the same time gather W1^T rows from the same region, for L2 reuse,
+// and a group's x tiles stay in L2). Two TMEM
 // accumulators alternate between tiles, so the epilogue of one tile overlaps
 // the main loop of the next; ring stages and parities follow one running
 // k-step counter across tiles.
@@ -174,7 +211,8 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
       // ahead and range-checked when they are used
       auto load_rows = [&](int tl, int *c) {
         const int tile = blockIdx.x + tl * gridDim.x;
-        const int chunk = tile / p.nb, b = tile % p.nb;
+        const TileAt ta = tile_at(tile, p.nb, p.nchunks, p.group);
+        const int chunk = ta.part, b = ta.b;
 #pragma unroll
         for (int i = 0; i < kRowIters; ++i)
           c[i] = tl < my_tiles ? __ldg(p.idx + static_cast<size_t>(b) * p.k +
@@ -218,7 +256,8 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
     bool ok = true;
     for (int tl = 0; tl < my_tiles && ok; ++tl) {
       const int tile = blockIdx.x + tl * gridDim.x;
-      const int chunk = tile / p.nb, b = tile % p.nb;
+      const TileAt ta = tile_at(tile, p.nb, p.nchunks, p.group);
+      const int chunk = ta.part, b = ta.b;
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         if (DENSE) {
           const int s = kg % SA;
@@ -315,7 +354,8 @@ __global__ void __launch_bounds__(UpCfg<BT>::kThreads, UpCfg<BT>::kCtasPerSm)
     const int ck = lane & 3, cq = lane >> 2;
     for (int tl = 0; tl < my_tiles; ++tl) {
       const int tile = blockIdx.x + tl * gridDim.x;
-      const int chunk = tile / p.nb, b = tile % p.nb;
+      const TileAt ta = tile_at(tile, p.nb, p.nchunks, p.group);
+      const int chunk = ta.part, b = ta.b;
       const int ab = tl & 1;
       const int j = chunk * 128 + r;
       bool valid_j = sparse ? (j < p.k) : (j < p.H);
@@ -581,7 +621,8 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
       // ahead and range-checked when they are used
       auto load_rows = [&](int tl, int *c) {
         const int tile = blockIdx.x + tl * gridDim.x;
-        const int chunk = tile / p.nb, b = tile % p.nb;
+        const TileAt ta = tile_at(tile, p.nb, nch, p.group);
+        const int chunk = ta.part, b = ta.b;
 #pragma unroll
         for (int i = 0; i < kRowIters; ++i)
           c[i] = tl < my_tiles ? __ldg(p.idx + static_cast<size_t>(b) * p.k +
@@ -624,7 +665,8 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
     bool ok = true;
     for (int tl = 0; tl < my_tiles && ok; ++tl) {
       const int tile = blockIdx.x + tl * gridDim.x;
-      const int chunk = tile / p.nb, b = tile % p.nb;
+      const TileAt ta = tile_at(tile, p.nb, nch, p.group);
+      const int chunk = ta.part, b = ta.b;
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         const int s = kg % S;
         if (!wait_warp(&empty[s], ((kg / S) & 1) ^ 1, p.status, abort_flag)) {
@@ -684,7 +726,8 @@ __global__ void __launch_bounds__(UpWideCfg<N>::kThreads, 1)
     uint32_t part_phase = 0;
     for (int tl = 0; tl < my_tiles; ++tl) {
       const int tile = blockIdx.x + tl * gridDim.x;
-      const int chunk = tile / p.nb, b = tile % p.nb;
+      const TileAt ta = tile_at(tile, p.nb, nch, p.group);
+      const int chunk = ta.part, b = ta.b;
       const int ab = tl & 1;
       const int nvalid = min(BT, p.T - b * BT);
       // hidden unit of column j = chunk * kN + 32 cc + lane, for all chunks cc
@@ -939,8 +982,9 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // slice-major across blocks: CTAs running at the same time share an N slice
-  // and sweep their (ascending) W2 rows in the same order (L2 reuse)
+  // grouped, slice-major in a group (tile_at): CTAs running at the same time
+  // share an N slice and sweep their (ascending) W2 rows in the same order (L2
+  // reuse), and a group's delta tiles stay in L2 while its slices are done
   if (warp < C::kProdWarps) {
     // gathered W2 rows: warp pw moves rows pw*R .. pw*R+R-1 (R = kRowsPerWarp) of each 64-row stage
     if (!DENSE) {
@@ -957,21 +1001,23 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
       // issued, into a register nothing reads until then (the loop body is
       // unrolled four times, so no move waits on a pending load); its range
       // is checked only when it is used.
+      // the tile's block and slice are worked out once per tile, not per stage
       int ltile = blockIdx.x, lkb = 0;                 // stage whose index is loaded next
+      const int32_t *lrow = p.idx + static_cast<size_t>(tile_at(ltile, p.nb, p.n_slices, p.group).b) * p.k;
       auto load_idx = [&]() -> int {
         int c = 0;
-        if (lane < kRowsPerWarp && ltile < ntiles)
-          c = __ldg(p.idx + static_cast<size_t>(ltile % p.nb) * p.k + min(lkb * kKStage + pw * kRowsPerWarp + lane, p.k - 1));
+        if (lane < kRowsPerWarp && ltile < ntiles) c = __ldg(lrow + min(lkb * kKStage + pw * kRowsPerWarp + lane, p.k - 1));
         if (++lkb == nk) {
           lkb = 0;
           ltile += gridDim.x;
+          if (ltile < ntiles) lrow = p.idx + static_cast<size_t>(tile_at(ltile, p.nb, p.n_slices, p.group).b) * p.k;
         }
         return c;
       };
       int tile = blockIdx.x, kb = 0;                   // stage whose copies are issued next
+      int n0 = tile_at(tile, p.nb, p.n_slices, p.group).part * BN;
       auto issue = [&](int kg, int c) -> bool {
         const int s = kg % SB;
-        const int n0 = (tile / p.nb) * BN;
         if (static_cast<unsigned>(c) >= static_cast<unsigned>(p.H)) {
           atomicCAS(p.status, kDevOk, kDevBadIndex);
           c = 0;
@@ -991,6 +1037,7 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
         if (++kb == nk) {
           kb = 0;
           tile += gridDim.x;
+          if (tile < ntiles) n0 = tile_at(tile, p.nb, p.n_slices, p.group).part * BN;
         }
         return true;
       };
@@ -1011,7 +1058,8 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
     int kg = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-      const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
+      const TileAt ta = tile_at(tile, p.nb, p.n_slices, p.group);
+      const int b = ta.b, n0 = ta.part * BN;
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         if (DENSE) {
           const int s = kg % SB;
@@ -1097,7 +1145,8 @@ __global__ void __launch_bounds__(DownCfg<BN>::kThreads, DownCfg<BN>::kCtasPerSm
     const bool accumulate = p.mode == kDownAccumulate;
     int tl = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
-      const int b = tile % p.nb, n0 = (tile / p.nb) * BN;
+      const TileAt ta = tile_at(tile, p.nb, p.n_slices, p.group);
+      const int b = ta.b, n0 = ta.part * BN;
       const int ab = tl % C::kAccs;
       if (!wait_warp(&acc_full[ab], (tl / C::kAccs) & 1, p.status, abort_flag)) break;
       tc_fence_after();
@@ -1228,7 +1277,9 @@ cudaError_t y_to_out(const MlpDownParams &p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_mlp_up_fp8(const MlpUpParams &p, const CUtensorMap &tm_x, cudaStream_t s) {
+cudaError_t launch_mlp_up_fp8(const MlpUpParams &p0, const CUtensorMap &tm_x, cudaStream_t s) {
+  MlpUpParams p = p0;
+  p.group = up_tile_group(p.nb, static_cast<int64_t>(p.Bt) * p.D);   // e4m3 x tiles
   if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
   if (p.Bt != 128 || p.mode != kUpDelta) return cudaErrorInvalidValue;
   using C = UpCfg<128>;
@@ -1243,7 +1294,9 @@ cudaError_t launch_mlp_up_fp8(const MlpUpParams &p, const CUtensorMap &tm_x, cud
   return cudaGetLastError();
 }
 
-cudaError_t launch_mlp_down_fp8(const MlpDownParams &p, const CUtensorMap &tm_a, cudaStream_t s) {
+cudaError_t launch_mlp_down_fp8(const MlpDownParams &p0, const CUtensorMap &tm_a, cudaStream_t s) {
+  MlpDownParams p = p0;
+  p.group = down_tile_group(p.nb, false, 0);
   if (p.nb <= 0) return cudaSuccess;
   if (p.k <= 0) return y_to_out(p, s);
   if (p.Bt != 128 || p.bn != 256 || p.mode != kDownAccumulate) return cudaErrorInvalidValue;
@@ -1259,7 +1312,9 @@ cudaError_t launch_mlp_down_fp8(const MlpDownParams &p, const CUtensorMap &tm_a,
   return cudaGetLastError();
 }
 
-cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s) {
+cudaError_t launch_mlp_up(const MlpUpParams &p0, const CUtensorMap &tm_w1t, const CUtensorMap &tm_x, cudaStream_t s) {
+  MlpUpParams p = p0;
+  p.group = up_tile_group(p.nb, static_cast<int64_t>(p.Bt) * p.D * 2);   // bf16 x tiles
   if (p.nb <= 0 || p.nchunks <= 0) return cudaSuccess;
   const bool dense = p.mode != kUpDelta;
   if (p.Bt == 128) return dense ? launch_up_wide<256, true>(p, tm_w1t, tm_x, s) : launch_up_t<128, false>(p, tm_w1t, tm_x, s);
@@ -1267,8 +1322,10 @@ cudaError_t launch_mlp_up(const MlpUpParams &p, const CUtensorMap &tm_w1t, const
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_mlp_down(const MlpDownParams &p, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
+cudaError_t launch_mlp_down(const MlpDownParams &p0, const CUtensorMap &tm_a, const CUtensorMap &tm_w2, bool dense,
                             cudaStream_t s) {
+  MlpDownParams p = p0;
+  p.group = down_tile_group(p.nb, dense, static_cast<int64_t>(p.krows) * p.Bt * 2);   // bf16 activation-cache tiles
   if (p.nb <= 0) return cudaSuccess;
   const int kext = dense ? p.krows : p.k;
   if (kext <= 0) return y_to_out(p, s);
