@@ -854,7 +854,7 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
-PROFILE_CASES = ("attn_delta", "mass_select", "mass_kept", "mlp")
+PROFILE_CASES = ("attn_delta", "mass_select", "mass_kept", "mlp", "topk_long")
 
 
 def run_profile_case(args):
@@ -864,13 +864,22 @@ def run_profile_case(args):
         its 24 heads (heads are independent, so per-launch traffic scales by 12). attn_delta runs the
         sparse step; mass_select the refresh without a mass tensor (the fused mass/top-k kernel keeps
         the rows in its L2 row buffers), mass_kept the refresh writing the mass [h][nb][T] to HBM.
-      mlp: the sparse MLP step (mlp_up, mlp_down) of the FLUX.1-dev 2304x1280 layer (T = 12032)."""
+      mlp: the sparse MLP step (mlp_up, mlp_down) of the FLUX.1-dev 2304x1280 layer (T = 12032).
+      topk_long: the top-k (k = 8316) of 2960 HunyuanVideo-length rows (118800) drawn as u^4, the bench's
+        `topk_hunyuan_attn_rows` row (1.41 GB)."""
     import torch
     from dynamic_column_sparse_b200 import chipmunk as cm
     cm.load_library()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if args.profile_case == "mlp":
+    if args.profile_case == "topk_long":
+        g = torch.Generator(device=dev).manual_seed(7)
+        hn, hk, hr = 118800, 8316, 148 * 20
+        hs = torch.rand((hr, hn), generator=g, device=dev) ** 4
+        for _ in range(args.steps):
+            cm.topk_cols(hs, hk)
+        info = {"rows": hr, "n": hn, "k": hk}
+    elif args.profile_case == "mlp":
         w = dict(FLUX, T=144 * 80 + 512, key="flux_2304x1280")
         L = Layer(w, dev, seed=99)
         for i in range(args.steps):

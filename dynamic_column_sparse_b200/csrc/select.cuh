@@ -19,14 +19,18 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 }
 
 // One shared-memory increment of hist[bin] for every lane that has `active`
-// set, one atomic per distinct bin of the warp (values that crowd into a few
-// bins would otherwise serialise on them). Warp-collective: every lane of the
-// warp must call it.
+// set. When all active lanes of the warp share one bin (values that crowd into
+// a few bins), a single atomic adds them all; otherwise each lane adds its own.
+// Warp-collective: every lane of the warp must call it.
 __device__ __forceinline__ void warp_hist_add(uint32_t *hist, uint32_t bin, bool active) {
   const unsigned am = __ballot_sync(0xffffffffu, active);
-  if (active) {
-    const unsigned peers = __match_any_sync(am, bin);
-    if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+  if (am == 0u) return;
+  const int leader = __ffs(am) - 1;
+  const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+  if (__all_sync(0xffffffffu, !active || bin == lb)) {
+    if ((threadIdx.x & 31) == static_cast<unsigned>(leader)) atomicAdd(&hist[lb], static_cast<uint32_t>(__popc(am)));
+  } else if (active) {
+    atomicAdd(&hist[bin], 1u);
   }
 }
 

@@ -339,15 +339,21 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
       }
       return true;
     };
-    // candidate L of the concatenated (index-ordered) list
-    auto cand_at = [&](int L, uint32_t &key, int32_t &idx) {
+    // candidate L of the concatenated (index-ordered) list lies in region
+    // cand_w(L), which holds candidates s_pref[w] .. s_pref[w+1]-1 from s_base[w] on
+    auto cand_w = [&](int L) -> int {
       int w = 0;
 #pragma unroll
       for (int step = kWarps / 2; step >= 1; step >>= 1)
         if (static_cast<uint32_t>(L) >= s_pref[w + step]) w += step;
-      const int j = static_cast<int>(s_base[w]) + (L - static_cast<int>(s_pref[w]));
-      key = ckey[j];
-      idx = cidx[j];
+      return w;
+    };
+    // whether buffer slot j holds a candidate (the radix passes need every
+    // candidate, in any order, so they walk the buffer itself)
+    auto slot_valid = [&](int j) -> bool {
+      if (s_base[kWarps - 1] == s_pref[kWarps - 1]) return j < static_cast<int>(s_pref[kWarps]);  // laid end to end
+      const int w = j / kRegion;
+      return j - w * kRegion < static_cast<int>(s_pref[w + 1] - s_pref[w]);
     };
     // radix passes over the first `count` keys of `keys` (or, with keys null,
     // over the candidates): from (prefix, mask, kk), the digits of passes
@@ -360,18 +366,12 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
         const int nbins = pass == 2 ? 1024 : 2048;
         for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
         __syncthreads();
-        for (int b0 = warp * 32; b0 < count; b0 += kThreads) {   // warp-uniform
+        const int span = keys ? count : kLongCap;
+        for (int b0 = warp * 32; b0 < span; b0 += kThreads) {   // warp-uniform
           const int L = b0 + lane;
-          uint32_t key = 0;
-          if (L < count) {
-            if (keys) {
-              key = keys[L];
-            } else {
-              int32_t unused;
-              cand_at(L, key, unused);
-            }
-          }
-          warp_hist_add(hist, (key >> shift) & static_cast<uint32_t>(nbins - 1), L < count && (key & mask) == prefix);
+          const bool valid = L < span && (keys ? true : slot_valid(L));
+          const uint32_t key = valid ? (keys ? keys[L] : ckey[L]) : 0u;
+          warp_hist_add(hist, (key >> shift) & static_cast<uint32_t>(nbins - 1), valid && (key & mask) == prefix);
         }
         __syncthreads();
         select_digit(hist, nbins, kk, warp_tot, s_digit, s_above);
@@ -390,11 +390,18 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
         const int first = base + tid * kItems;
         uint32_t keys[kItems];
         int32_t ids[kItems];
+        int w = first < count ? cand_w(first) : 0;   // found once, then walked forwards
 #pragma unroll
         for (int e = 0; e < kItems; ++e) {
           keys[e] = 0u;
           ids[e] = 0;
-          if (first + e < count) cand_at(first + e, keys[e], ids[e]);
+          const int L = first + e;
+          if (L < count) {
+            while (static_cast<uint32_t>(L) >= s_pref[w + 1]) ++w;
+            const int j = static_cast<int>(s_base[w]) + (L - static_cast<int>(s_pref[w]));
+            keys[e] = ckey[j];
+            ids[e] = cidx[j];
+          }
         }
         compact_tile(keys, first, count, tau, kk, k, run_gt, run_eq, warp_tot,
                      [&](uint32_t pos, int e) { dst[pos] = ids[e]; });
@@ -475,15 +482,13 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(const TopkParams p)
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
       const int shift = pass == 0 ? 10 : 0;
-      const int count = static_cast<int>(s_pref[kWarps]);
       for (int i = tid; i < 1024; i += kThreads) hist[i] = 0;
       __syncthreads();
-      for (int b0 = warp * 32; b0 < count; b0 += kThreads) {   // warp-uniform
+      for (int b0 = warp * 32; b0 < kLongCap; b0 += kThreads) {   // warp-uniform
         const int L = b0 + lane;
-        uint32_t key = 0;
-        int32_t unused;
-        if (L < count) cand_at(L, key, unused);
-        warp_hist_add(hist, (key >> shift) & 1023u, L < count && (key & mask) == prefix);
+        const bool valid = slot_valid(L);
+        const uint32_t key = valid ? ckey[L] : 0u;
+        warp_hist_add(hist, (key >> shift) & 1023u, valid && (key & mask) == prefix);
       }
       __syncthreads();
       select_digit(hist, 1024, kk, warp_tot, s_digit, s_above);
