@@ -20,8 +20,11 @@
 // fit, the regions are laid end to end after a counting pass. A row whose
 // candidates do not fit at all, or that is not 16-byte aligned, falls back to
 // the general path that re-reads the row from global memory for every radix
-// pass. Histogram increments are aggregated per warp and bin, so scores that
-// crowd into a few bins do not serialise on one shared-memory atomic each.
+// pass. The radix passes over the candidates walk the warps' regions as they
+// lie (they need every candidate, in any order); the compaction, which needs
+// index order, finds each thread's region once and walks forwards. A warp
+// whose active lanes all fall in one histogram bin (scores that crowd into a
+// few bins) adds them with one shared-memory atomic.
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
