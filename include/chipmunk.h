@@ -223,7 +223,7 @@ CHIPMUNK_API chipmunk_status chipmunk_mlp_delta_down(const chipmunk_mlp_args *a,
 
 /*
  * chipmunk_mlp_delta_noalloc - the sparse MLP step for callers that cannot
- * allocate device memory. No counterpart in the paper: the post describes the
+ * allocate device memory. No counterpart in the blog post, which describes the
  * method, not how its scratch memory is obtained.
  *
  * Some callers can't call cudaMalloc: a host framework that owns all device
